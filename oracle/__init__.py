@@ -39,6 +39,7 @@ def lib():
         L.oracle_e4m3_value.restype = C.c_double
         L.oracle_e4m3_rne_satfinite.argtypes = [C.c_double]
         L.oracle_e4m3_rne_satfinite.restype = C.c_uint8
+        L.oracle_to_bf16.argtypes = [vp, i64, vp]
         L.oracle_pack_groupwise.argtypes = [i32, vp, i64, i64, vp, vp, vp]
         L.oracle_pack_fp8_row.argtypes = [vp, i64, i64, vp, vp]
         L.oracle_decode_mxfp8.argtypes = [vp, vp, i64, i64, vp]
@@ -48,7 +49,7 @@ def lib():
         L.oracle_quantize_act.argtypes = [vp, i64, i64, vp, vp]
         L.oracle_group_sums.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp]
         L.oracle_gemm_a8.argtypes = [i32, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, i32]
-        for name in ("oracle_pack_groupwise", "oracle_pack_fp8_row", "oracle_decode_mxfp8",
+        for name in ("oracle_to_bf16", "oracle_pack_groupwise", "oracle_pack_fp8_row", "oracle_decode_mxfp8",
                      "oracle_decode_mlx_affine", "oracle_dequant", "oracle_gemv",
                      "oracle_quantize_act", "oracle_group_sums", "oracle_gemm_a8"):
             getattr(L, name).restype = C.c_int
@@ -126,7 +127,8 @@ def pack(fmt, w):
         _check(lib().oracle_pack_groupwise(fmt, _p(w), n, k, _p(codes), _p(hib), _p(scales)),
                "pack_groupwise")
     elif fmt == BF16:
-        codes = np.array([[bf16_rne(float(v)) for v in row] for row in w], np.uint16)
+        codes = np.zeros((n, k), np.uint16)
+        _check(lib().oracle_to_bf16(_p(w), n * k, _p(codes)), "to_bf16")
         scales = None
     else:
         raise ValueError(fmt)

@@ -230,6 +230,12 @@ uint16_t oracle_bf16_rne(double v) { return bf16_rne(v); }
 double oracle_e4m3_value(uint8_t c) { return e4m3_value(c); }
 uint8_t oracle_e4m3_rne_satfinite(double v) { return e4m3_rne_satfinite(v); }
 
+// BF16 re-encode of float32 values (the QLIN_BF16 target format).
+int oracle_to_bf16(const float* v, int64_t count, uint16_t* out) {
+  for (int64_t i = 0; i < count; ++i) out[i] = bf16_rne((double)v[i]);
+  return 0;
+}
+
 // ---- groupwise integer packing --------------------------------------------
 // [NVFP4] "What is in the file": Q4/Q5/Q8 grouped, FP16 scales.
 // [RTX5080] "Quantization profile": Q4G64_F16S, Q5G64_F16S (group 64).

@@ -1,0 +1,235 @@
+// C ABI entry points (include/qlin.h): argument validation on the host, then
+// dispatch to the kernel launchers.  Nothing here allocates device memory.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "qlin_internal.cuh"
+
+namespace qlin {
+
+size_t gemv_cc_workspace_bytes(const qlin_weights& w, int64_t t);
+int launch_gemv_cc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
+                   const Exec& ex, float* acc_ws);
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int make_exec(const qlin_exec* e, Exec* out) {
+  out->stream = e ? (cudaStream_t)e->stream : (cudaStream_t)0;
+  out->dev_status = e ? e->dev_status : nullptr;
+  out->workspace = e ? e->workspace : nullptr;
+  out->workspace_bytes = e ? e->workspace_bytes : 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLIN_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&out->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return QLIN_ERR_CUDA;
+  if (out->workspace && !aligned16(out->workspace)) return QLIN_ERR_INVALID_ARG;
+  return QLIN_OK;
+}
+
+int group_of(int fmt) {
+  switch (fmt) {
+    case QLIN_Q4_G64:
+    case QLIN_Q5_G64:
+    case QLIN_FP8_ROW:
+    case QLIN_BF16:
+      return 64;
+    case QLIN_Q8_G32:
+      return 32;
+    default:
+      return 0;
+  }
+}
+
+int sizes_of(int fmt, int64_t n, int64_t k, size_t* c, size_t* h, size_t* s) {
+  int g = group_of(fmt);
+  if (g == 0 || n <= 0 || k <= 0 || k % g != 0) return QLIN_ERR_INVALID_ARG;
+  size_t cb = 0, hb = 0, sb = 0;
+  switch (fmt) {
+    case QLIN_Q4_G64: cb = (size_t)n * (k / 2); sb = (size_t)n * (k / 64) * 2; break;
+    case QLIN_Q5_G64: cb = (size_t)n * (k / 2); hb = (size_t)n * (k / 8); sb = (size_t)n * (k / 64) * 2; break;
+    case QLIN_Q8_G32: cb = (size_t)n * k; sb = (size_t)n * (k / 32) * 2; break;
+    case QLIN_FP8_ROW: cb = (size_t)n * k; sb = (size_t)n * 2; break;
+    case QLIN_BF16: cb = (size_t)n * k * 2; break;
+  }
+  if (c) *c = cb;
+  if (h) *h = hb;
+  if (s) *s = sb;
+  return QLIN_OK;
+}
+
+int check_weights(const qlin_weights* w) {
+  if (!w) return QLIN_ERR_INVALID_ARG;
+  size_t c, h, s;
+  int rc = sizes_of(w->fmt, w->n, w->k, &c, &h, &s);
+  if (rc) return rc;
+  if (!w->codes || !aligned16(w->codes)) return QLIN_ERR_INVALID_ARG;
+  if (h && (!w->hibits || !aligned16(w->hibits))) return QLIN_ERR_INVALID_ARG;
+  if (s && (!w->scales || !aligned16(w->scales))) return QLIN_ERR_INVALID_ARG;
+  return QLIN_OK;
+}
+
+}  // namespace
+
+int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                   uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+  });
+  if (!g_encode) return QLIN_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QLIN_OK : QLIN_ERR_CUDA;
+}
+
+size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
+  (void)num_sms;
+  return gemv_cc_workspace_bytes(w, t);
+}
+
+int launch_gemv(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
+                const Exec& ex) {
+  return launch_gemv_cc(w, x, t, y, y_dtype, ex, (float*)ex.workspace);
+}
+
+}  // namespace qlin
+
+using namespace qlin;
+
+extern "C" {
+
+const char* qlin_status_string(int status) {
+  switch (status) {
+    case QLIN_OK: return "ok";
+    case QLIN_ERR_INVALID_ARG: return "invalid argument";
+    case QLIN_ERR_UNSUPPORTED: return "unsupported request";
+    case QLIN_ERR_NOT_PERMITTED: return "int8 route not permitted for these weights";
+    case QLIN_ERR_CUDA: return "CUDA error";
+    case QLIN_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case QLIN_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int qlin_packed_bytes(int fmt, int64_t n, int64_t k, size_t* codes_bytes, size_t* hibits_bytes,
+                      size_t* scales_bytes) {
+  return sizes_of(fmt, n, k, codes_bytes, hibits_bytes, scales_bytes);
+}
+
+int qlin_pack_weights(int src_kind, const void* src, const void* src_aux0, const void* src_aux1,
+                      const qlin_weights* dst, const qlin_exec* ex) {
+  int rc = check_weights(dst);
+  if (rc) return rc;
+  if (!src || !aligned16(src)) return QLIN_ERR_INVALID_ARG;
+  switch (src_kind) {
+    case QLIN_SRC_F32:
+    case QLIN_SRC_BF16:
+      break;
+    case QLIN_SRC_MXFP8:
+      if (dst->k % 32 || !src_aux0 || !aligned16(src_aux0)) return QLIN_ERR_INVALID_ARG;
+      break;
+    case QLIN_SRC_MLX_AFFINE8:
+      if (dst->k % 128 || !src_aux0 || !src_aux1 || !aligned16(src_aux0) || !aligned16(src_aux1))
+        return QLIN_ERR_INVALID_ARG;
+      break;
+    default:
+      return QLIN_ERR_INVALID_ARG;
+  }
+  Exec e;
+  if ((rc = make_exec(ex, &e))) return rc;
+  return launch_pack(src_kind, src, src_aux0, src_aux1, *dst, e);
+}
+
+int qlin_decode_mxfp8(const uint32_t* words, const uint8_t* scales, int64_t rows, int64_t cols,
+                      uint16_t* out_bf16, const qlin_exec* ex) {
+  if (!words || !scales || !out_bf16 || rows <= 0 || cols <= 0 || cols % 32) return QLIN_ERR_INVALID_ARG;
+  if (!aligned16(words) || !aligned16(out_bf16)) return QLIN_ERR_INVALID_ARG;
+  Exec e;
+  int rc = make_exec(ex, &e);
+  if (rc) return rc;
+  return launch_decode_mxfp8(words, scales, rows, cols, out_bf16, e);
+}
+
+int qlin_quantize_act(const uint16_t* x_bf16, int64_t t, int64_t k, int8_t* xq, float* xs,
+                      const qlin_exec* ex) {
+  if (!x_bf16 || !xq || !xs || t <= 0 || k <= 0 || k % 64) return QLIN_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(xq) || !aligned16(xs)) return QLIN_ERR_INVALID_ARG;
+  Exec e;
+  int rc = make_exec(ex, &e);
+  if (rc) return rc;
+  return launch_quantize_act(x_bf16, t, k, xq, xs, e);
+}
+
+int qlin_gemv_workspace_bytes(const qlin_weights* w, int64_t t, size_t* bytes) {
+  int rc = check_weights(w);
+  if (rc) return rc;
+  if (!bytes || t <= 0) return QLIN_ERR_INVALID_ARG;
+  Exec e;
+  if ((rc = make_exec(nullptr, &e))) return rc;
+  *bytes = gemv_workspace_bytes(*w, t, e.num_sms);
+  return QLIN_OK;
+}
+
+int qlin_gemv(const qlin_weights* w, const uint16_t* x_bf16, int64_t t, void* y, int y_dtype,
+              const qlin_exec* ex) {
+  int rc = check_weights(w);
+  if (rc) return rc;
+  if (!x_bf16 || !y || t <= 0 || !aligned16(x_bf16) || !aligned16(y)) return QLIN_ERR_INVALID_ARG;
+  if (y_dtype != QLIN_OUT_BF16 && y_dtype != QLIN_OUT_F32) return QLIN_ERR_INVALID_ARG;
+  if (w->fmt != QLIN_BF16 && t > 64) return QLIN_ERR_UNSUPPORTED;
+  Exec e;
+  if ((rc = make_exec(ex, &e))) return rc;
+  size_t need = gemv_workspace_bytes(*w, t, e.num_sms);
+  if (need > e.workspace_bytes || (need && !e.workspace)) return QLIN_ERR_WORKSPACE;
+  return launch_gemv(*w, x_bf16, t, y, y_dtype, e);
+}
+
+int qlin_gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, size_t* bytes) {
+  if (!bytes || t <= 0 || n <= 0 || k <= 0 || k % 64) return QLIN_ERR_INVALID_ARG;
+  *bytes = gemm_a8_workspace_bytes(t, n, k, 0);
+  return QLIN_OK;
+}
+
+int qlin_gemm_a8(const qlin_weights* w, const uint16_t* x_bf16, const int8_t* xq, const float* xs,
+                 int64_t t, void* y, int y_dtype, uint32_t flags, int32_t* group_sums_dbg,
+                 const qlin_exec* ex) {
+  int rc = check_weights(w);
+  if (rc) return rc;
+  if (w->fmt != QLIN_Q4_G64 && w->fmt != QLIN_Q5_G64) return QLIN_ERR_UNSUPPORTED;
+  if (!(w->flags & QLIN_ALLOW_A8)) return QLIN_ERR_NOT_PERMITTED;
+  if (w->fmt == QLIN_Q5_G64 && w->k % 128) return QLIN_ERR_UNSUPPORTED;
+  if (t <= 0 || !y || !aligned16(y)) return QLIN_ERR_INVALID_ARG;
+  if (y_dtype != QLIN_OUT_BF16 && y_dtype != QLIN_OUT_F32) return QLIN_ERR_INVALID_ARG;
+  const bool fused = x_bf16 != nullptr;
+  if (fused == (xq != nullptr || xs != nullptr)) return QLIN_ERR_INVALID_ARG;
+  if (fused && !aligned16(x_bf16)) return QLIN_ERR_INVALID_ARG;
+  if (!fused && (!xq || !xs || !aligned16(xq) || !aligned16(xs))) return QLIN_ERR_INVALID_ARG;
+  if ((flags & QLIN_DEBUG_GROUP_SUMS) && !group_sums_dbg) return QLIN_ERR_INVALID_ARG;
+  if (t > (int64_t)INT32_MAX || w->n > (int64_t)INT32_MAX || w->k > (int64_t)INT32_MAX)
+    return QLIN_ERR_UNSUPPORTED;
+  Exec e;
+  if ((rc = make_exec(ex, &e))) return rc;
+  if (fused) {
+    size_t need = gemm_a8_workspace_bytes(t, w->n, w->k, e.num_sms);
+    if (need > e.workspace_bytes || !e.workspace) return QLIN_ERR_WORKSPACE;
+  }
+  return launch_gemm_a8(*w, x_bf16, xq, xs, t, y, y_dtype, flags, group_sums_dbg, e);
+}
+
+}  // extern "C"

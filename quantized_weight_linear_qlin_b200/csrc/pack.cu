@@ -1,0 +1,258 @@
+// Weight packing and source decoding kernels (offline converter steps run on
+// the device).  All of it is bit-exact by construction: IEEE division
+// (__fdiv_rn), round-to-nearest-even conversions and fused multiply-adds only
+// where the definition has one.
+//
+// Sources: "Qwen3.8-27B MXFP8-CRACK -- NInfer artifact", "How it was built"
+// (step 1 MXFP8, step 2 MLX affine int8); "Qwen3.8-27B EfficientThink-
+// Uncensored FP8 for NInfer", "Conversion and verification" (fp8_row_maxabs);
+// "Qwen3.8-27B for NInfer -- RTX 5080 16 GB", "Quantization profile"
+// (Q4G64_F16S, Q5G64_F16S); "...NVFP4-NInferV3", "What is in the file" (Q8).
+#include "qlin_internal.cuh"
+
+namespace qlin {
+namespace {
+
+// ---- source element -> FP32 value -----------------------------------------
+struct Src {
+  int kind;
+  const void* src;
+  const void* aux0;
+  const void* aux1;
+  int64_t k;
+};
+
+// E4M3 byte -> float (exact; via the hardware E4M3 -> f16 conversion).
+__device__ __forceinline__ float e4m3_to_float(uint8_t c) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// 2^(b-127) as a float (b in 0..254; b = 0 is the subnormal 2^-127).
+__device__ __forceinline__ float ue8m0_to_float(uint32_t b) {
+  return b == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(b << 23);
+}
+
+// MXFP8 element -> bfloat16 bits (exact product, one BF16 rounding).
+__device__ __forceinline__ uint16_t mxfp8_to_bf16(uint8_t c, uint32_t b) {
+  if ((c & 0x7F) == 0x7F || b == 255) return (uint16_t)(0x7FC0 | ((c & 0x80) << 8));
+  float v = __fmul_rn(e4m3_to_float(c), ue8m0_to_float(b));
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
+  return __uint_as_float((uint32_t)h << 16);
+}
+
+__device__ __forceinline__ float source_value(const Src& s, int64_t r, int64_t c) {
+  switch (s.kind) {
+    case QLIN_SRC_F32:
+      return ((const float*)s.src)[r * s.k + c];
+    case QLIN_SRC_BF16:
+      return bf16_bits_to_float(((const uint16_t*)s.src)[r * s.k + c]);
+    case QLIN_SRC_MXFP8: {
+      uint32_t w = ((const uint32_t*)s.src)[r * (s.k / 4) + c / 4];
+      uint8_t code = (uint8_t)(w >> (8 * (c & 3)));
+      uint32_t b = ((const uint8_t*)s.aux0)[r * (s.k / 32) + c / 32];
+      return bf16_bits_to_float(mxfp8_to_bf16(code, b));
+    }
+    default: {  // MLX affine int8: one FP32 fma, then BF16
+      uint8_t q = ((const uint8_t*)s.src)[r * s.k + c];
+      int64_t gi = r * (s.k / 128) + c / 128;
+      float sc = __half2float(((const __half*)s.aux0)[gi]);
+      float bi = __half2float(((const __half*)s.aux1)[gi]);
+      float v = __fmaf_rn((float)q, sc, bi);
+      return __bfloat162float(__float2bfloat16_rn(v));
+    }
+  }
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_or(uint32_t v, int width) {
+  for (int o = 1; o < width; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ---- Q4 / Q5 group-64: one warp per (row, group); lane l owns elements 2l, 2l+1.
+template <int BITS>
+__global__ void pack_q4q5_kernel(Src s, int64_t n, uint8_t* codes, uint8_t* hibits,
+                                 __half* scales) {
+  constexpr float QMAX = BITS == 4 ? 7.0f : 15.0f;
+  constexpr int OFF = BITS == 4 ? 8 : 16;
+  const int64_t ng = s.k / 64;
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (item >= n * ng) return;
+  const int64_t r = item / ng, g = item % ng;
+  const int64_t e0 = g * 64 + 2 * lane;
+  float v0 = source_value(s, r, e0), v1 = source_value(s, r, e0 + 1);
+  float a = warp_max(fmaxf(fabsf(v0), fabsf(v1)));
+  __half s16 = __float2half_rn(__fdiv_rn(a, QMAX));
+  float sc = __half2float(s16);
+  int q0 = 0, q1 = 0;
+  if (sc != 0.0f) {
+    q0 = (int)fminf(fmaxf(rintf(__fdiv_rn(v0, sc)), -QMAX - 1.0f), QMAX);
+    q1 = (int)fminf(fmaxf(rintf(__fdiv_rn(v1, sc)), -QMAX - 1.0f), QMAX);
+  }
+  uint32_t u0 = (uint32_t)(q0 + OFF), u1 = (uint32_t)(q1 + OFF);
+  // nibble word: lanes 4j..4j+3 cover word j; lane's s = lane & 3
+  int sl = lane & 3;
+  uint32_t part = ((u0 & 0xF) << (4 * sl)) | ((u1 & 0xF) << (16 + 4 * sl));
+  uint32_t word = warp_or(part, 4);
+  if (sl == 0) {
+    uint32_t* row = (uint32_t*)(codes + r * (s.k / 2));
+    row[(e0 >> 3)] = word;
+  }
+  if (BITS == 5) {
+    // element e (in group) = 2*lane + o; word h = lane / 16 ; jj = (lane % 16) / 4 ; s = lane % 4
+    int jj = (lane & 15) >> 2;
+    uint32_t hp = (((u0 >> 4) & 1u) << (4 * jj + sl)) | (((u1 >> 4) & 1u) << (16 + 4 * jj + sl));
+    uint32_t hw = warp_or(hp, 16);
+    if ((lane & 15) == 0) {
+      uint32_t* hrow = (uint32_t*)(hibits + r * (s.k / 8));
+      hrow[(e0 >> 5)] = hw;
+    }
+  }
+  if (lane == 0) scales[r * ng + g] = s16;
+}
+
+// ---- Q8 group-32: one warp per (row, group); lane l owns element l.
+__global__ void pack_q8_kernel(Src s, int64_t n, int8_t* codes, __half* scales) {
+  const int64_t ng = s.k / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (item >= n * ng) return;
+  const int64_t r = item / ng, g = item % ng;
+  const int64_t e = g * 32 + lane;
+  float v = source_value(s, r, e);
+  float a = warp_max(fabsf(v));
+  __half s16 = __float2half_rn(__fdiv_rn(a, 127.0f));
+  float sc = __half2float(s16);
+  int q = 0;
+  if (sc != 0.0f) q = (int)fminf(fmaxf(rintf(__fdiv_rn(v, sc)), -128.0f), 127.0f);
+  codes[r * s.k + e] = (int8_t)q;
+  if (lane == 0) scales[r * ng + g] = s16;
+}
+
+// ---- FP8 row (fp8_row_maxabs): one block per row.
+__global__ void pack_fp8_row_kernel(Src s, int64_t n, uint8_t* codes, __nv_bfloat16* scales) {
+  __shared__ float red[32];
+  const int64_t r = blockIdx.x;
+  float a = 0.0f;
+  for (int64_t c = threadIdx.x; c < s.k; c += blockDim.x) a = fmaxf(a, fabsf(source_value(s, r, c)));
+  a = warp_max(a);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < blockDim.x / 32 ? red[threadIdx.x] : 0.0f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  a = red[0];
+  __nv_bfloat16 sc16 = __float2bfloat16_rn(__fdiv_rn(a, 448.0f));
+  float sc = __bfloat162float(sc16);
+  for (int64_t c = threadIdx.x; c < s.k; c += blockDim.x) {
+    uint8_t code = 0;
+    if (sc != 0.0f)
+      code = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(source_value(s, r, c), sc), __NV_SATFINITE,
+                                            __NV_E4M3);
+    codes[r * s.k + c] = code;
+  }
+  if (threadIdx.x == 0) scales[r] = sc16;
+}
+
+// ---- BF16 target: BF16_rne of the source value.
+__global__ void pack_bf16_kernel(Src s, int64_t n, uint16_t* out) {
+  int64_t total = n * s.k;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t r = i / s.k, c = i % s.k;
+    out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(source_value(s, r, c)));
+  }
+}
+
+// ---- MXFP8 -> BF16 streaming decode: each thread turns one 16-byte chunk of
+// words (16 elements) into 32 bytes of BF16.
+__global__ void decode_mxfp8_kernel(const uint4* __restrict__ words, const uint8_t* __restrict__ sc,
+                                    int64_t rows, int64_t cols, uint4* __restrict__ out) {
+  const int64_t chunks_per_row = cols / 16;
+  const int64_t total = rows * chunks_per_row;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t r = i / chunks_per_row, ch = i % chunks_per_row;
+    uint4 w = __ldcs(words + i);
+    uint32_t b = sc[r * (cols / 32) + (ch >> 1)];
+    uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint16_t h0 = mxfp8_to_bf16((uint8_t)(wv[j]), b);
+      uint16_t h1 = mxfp8_to_bf16((uint8_t)(wv[j] >> 8), b);
+      uint16_t h2 = mxfp8_to_bf16((uint8_t)(wv[j] >> 16), b);
+      uint16_t h3 = mxfp8_to_bf16((uint8_t)(wv[j] >> 24), b);
+      o[2 * j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+      o[2 * j + 1] = (uint32_t)h2 | ((uint32_t)h3 << 16);
+    }
+    __stcs(out + 2 * i, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcs(out + 2 * i + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  }
+}
+
+}  // namespace
+
+int launch_pack(int src_kind, const void* src, const void* aux0, const void* aux1,
+                const qlin_weights& dst, const Exec& ex) {
+  Src s{src_kind, src, aux0, aux1, dst.k};
+  const int64_t n = dst.n;
+  switch (dst.fmt) {
+    case QLIN_Q4_G64:
+    case QLIN_Q5_G64: {
+      int64_t items = n * (dst.k / 64);
+      int64_t blocks = (items + 7) / 8;
+      if (dst.fmt == QLIN_Q4_G64)
+        pack_q4q5_kernel<4><<<(unsigned)blocks, 256, 0, ex.stream>>>(s, n, (uint8_t*)dst.codes,
+                                                                    nullptr, (__half*)dst.scales);
+      else
+        pack_q4q5_kernel<5><<<(unsigned)blocks, 256, 0, ex.stream>>>(
+            s, n, (uint8_t*)dst.codes, (uint8_t*)dst.hibits, (__half*)dst.scales);
+      break;
+    }
+    case QLIN_Q8_G32: {
+      int64_t items = n * (dst.k / 32);
+      pack_q8_kernel<<<(unsigned)((items + 7) / 8), 256, 0, ex.stream>>>(
+          s, n, (int8_t*)dst.codes, (__half*)dst.scales);
+      break;
+    }
+    case QLIN_FP8_ROW:
+      pack_fp8_row_kernel<<<(unsigned)n, 256, 0, ex.stream>>>(s, n, (uint8_t*)dst.codes,
+                                                              (__nv_bfloat16*)dst.scales);
+      break;
+    case QLIN_BF16: {
+      int64_t total = n * dst.k;
+      int64_t blocks = (total + 255) / 256;
+      if (blocks > (int64_t)ex.num_sms * 32) blocks = (int64_t)ex.num_sms * 32;
+      pack_bf16_kernel<<<(unsigned)blocks, 256, 0, ex.stream>>>(s, n, (uint16_t*)dst.codes);
+      break;
+    }
+    default:
+      return QLIN_ERR_INVALID_ARG;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_decode_mxfp8(const uint32_t* words, const uint8_t* scales, int64_t rows, int64_t cols,
+                        uint16_t* out, const Exec& ex) {
+  int64_t total = rows * (cols / 16);
+  int64_t blocks = (total + 255) / 256;
+  int64_t cap = (int64_t)ex.num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  decode_mxfp8_kernel<<<(unsigned)blocks, 256, 0, ex.stream>>>((const uint4*)words, scales, rows,
+                                                               cols, (uint4*)out);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace qlin

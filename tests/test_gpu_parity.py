@@ -1,0 +1,335 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Bit-exact for codes, scales, decodes, activation codes
+and int32 group sums; within the stated tolerances for FP32/BF16 outputs:
+|y - y_ref| <= 1e-3 * sum|w||x| (BF16 route) and <= 5e-6 * sum|q ws||qa as|
+(int8 route, FP32 output before rounding); a BF16 output may differ by one
+more half BF16 ulp of |y_ref| (its own rounding: half an ulp is at most 2^-8 of the value)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_weight_linear_qlin_b200 as q
+import synth
+
+pytestmark = pytest.mark.gpu
+
+FMTS = {"q4": q.Q4_G64, "q5": q.Q5_G64, "q8": q.Q8_G32, "fp8": q.FP8_ROW, "bf16": q.BF16}
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from quantized_weight_linear_qlin_b200 import _build
+    _build.build()
+    q.lib()
+
+
+def bits16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_value(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def gpu_packed_to_numpy(pw):
+    n, k = pw.n, pw.k
+    cdt, cshape, hshape, sdt, sshape = oracle.packed_shapes(pw.fmt, n, k)
+    codes = pw.codes.cpu().numpy().view(cdt).reshape(cshape)
+    hib = pw.hibits.cpu().numpy().reshape(hshape) if hshape else None
+    sc = pw.scales.cpu().numpy().view(sdt).reshape(sshape) if sshape else None
+    return {"fmt": pw.fmt, "n": n, "k": k, "codes": codes, "hibits": hib, "scales": sc}
+
+
+def pack_gpu(fmt, w_dev, allow_a8=False, src_kind=q.SRC_F32, aux0=None, aux1=None):
+    n, k = w_dev.shape[0], (w_dev.shape[1] * (4 if src_kind == q.SRC_MXFP8 else 1))
+    pw = q.PackedWeights(fmt, n, k, device=DEV, allow_a8=allow_a8)
+    q.qlin_pack_weights(src_kind, w_dev, pw, aux0=aux0, aux1=aux1)
+    return pw
+
+
+def assert_packed_equal(pw, ref):
+    got = gpu_packed_to_numpy(pw)
+    for key in ("codes", "hibits", "scales"):
+        if ref[key] is None:
+            continue
+        assert np.array_equal(got[key], ref[key]), key
+
+
+# ---------------------------------------------------------------------------
+# packing and decoding: bit-exact
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("fmt", list(FMTS))
+@pytest.mark.parametrize("shape", [(200, 320), (129, 1024)])
+def test_pack_from_f32_bit_exact(fmt, shape):
+    n, k = shape
+    w = synth.weights_f32(n, k, seed=100 + n)
+    w[3, :64] = 0.0          # an all-zero group
+    w[5] = 0.0               # an all-zero row (FP8 row scale 0)
+    w[7, 10] = 1e-30         # a tiny value next to a large one
+    w[8, :] *= 1e3
+    ref = oracle.pack(FMTS[fmt], w.numpy())
+    pw = pack_gpu(FMTS[fmt], w.to(DEV))
+    torch.cuda.synchronize()
+    assert_packed_equal(pw, ref)
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q5", "q8", "fp8"])
+def test_pack_from_bf16_bit_exact(fmt):
+    w = synth.weights_f32(96, 512, seed=7).to(torch.bfloat16)
+    ref = oracle.pack(FMTS[fmt], w.float().numpy())
+    pw = pack_gpu(FMTS[fmt], w.to(DEV).view(torch.int16), src_kind=q.SRC_BF16)
+    torch.cuda.synchronize()
+    assert_packed_equal(pw, ref)
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q5", "q8", "fp8", "bf16"])
+def test_pack_from_mxfp8_bit_exact(fmt):
+    rows, cols = 64, 512
+    words, scales = synth.mxfp8_source(rows, cols, seed=11)
+    dec = oracle.decode_mxfp8(words.numpy().view(np.uint32), scales.numpy(), rows, cols)
+    ref = oracle.pack(FMTS[fmt], bf16_value(dec).astype(np.float32))
+    pw = pack_gpu(FMTS[fmt], words.to(DEV), src_kind=q.SRC_MXFP8, aux0=scales.to(DEV))
+    torch.cuda.synchronize()
+    assert_packed_equal(pw, ref)
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q8", "bf16"])
+def test_pack_from_mlx_affine_bit_exact(fmt):
+    rows, cols = 48, 384
+    qq, s16, b16 = synth.mlx_affine_source(rows, cols, seed=13)
+    dec = oracle.decode_mlx_affine(qq.numpy(), s16.numpy().view(np.uint16), b16.numpy().view(np.uint16),
+                                   rows, cols)
+    ref = oracle.pack(FMTS[fmt], bf16_value(dec).astype(np.float32))
+    pw = q.PackedWeights(FMTS[fmt], rows, cols, device=DEV)
+    q.qlin_pack_weights(q.SRC_MLX_AFFINE8, qq.to(DEV), pw, aux0=s16.to(DEV), aux1=b16.to(DEV))
+    torch.cuda.synchronize()
+    assert_packed_equal(pw, ref)
+
+
+def test_decode_mxfp8_exhaustive_bit_exact():
+    # every code at every block exponent, NaNs included
+    codes = np.tile(np.arange(256, dtype=np.uint8), 256).reshape(256, 256)
+    words = codes.view(np.uint32).reshape(256, 64)
+    scales = np.repeat(np.arange(256, dtype=np.uint8)[:, None], 8, axis=1)
+    ref = oracle.decode_mxfp8(words, scales, 256, 256)
+    out = torch.empty(256, 256, dtype=torch.int16, device=DEV)
+    q.qlin_decode_mxfp8(torch.from_numpy(words.view(np.int32)).to(DEV),
+                        torch.from_numpy(scales).to(DEV), 256, 256, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), ref)
+
+
+def test_decode_mxfp8_full_size_bit_exact():
+    rows, cols = 5120, 17408
+    words, scales = synth.mxfp8_source(rows, cols, seed=synth.seed_for(2, 1), device=DEV)
+    out = torch.empty(rows, cols, dtype=torch.int16, device=DEV)
+    q.qlin_decode_mxfp8(words, scales, rows, cols, out)
+    sel = torch.arange(0, rows, 97)
+    ref = oracle.decode_mxfp8(words[sel].cpu().numpy().view(np.uint32), scales[sel].cpu().numpy(),
+                              len(sel), cols)
+    torch.cuda.synchronize()
+    assert np.array_equal(out[sel.to(DEV)].cpu().numpy().view(np.uint16), ref)
+
+
+# ---------------------------------------------------------------------------
+# activation quantizer: bit-exact
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(1, 64), (37, 320), (130, 5120), (5, 17408)])
+def test_quantize_act_bit_exact(shape):
+    t, k = shape
+    x = synth.activations_bf16(t, k, seed=t + k)
+    xf = x.float()
+    xf[0, :64] = 0.0                     # zero group
+    if t > 2:
+        xf[2, 64:128] = 3.0e38           # huge values
+        xf[1, :64] = 1e-38               # tiny values
+    x = xf.to(torch.bfloat16)
+    qa_ref, as_ref = oracle.quantize_act(bits16(x))
+    xq = torch.empty(t, k, dtype=torch.int8, device=DEV)
+    xs = torch.empty(t, k // 64, dtype=torch.float32, device=DEV)
+    q.qlin_quantize_act(x.to(DEV), xq, xs)
+    torch.cuda.synchronize()
+    assert np.array_equal(xq.cpu().numpy(), qa_ref)
+    assert np.array_equal(xs.cpu().numpy().view(np.uint32), as_ref.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# BF16-route GEMV
+# ---------------------------------------------------------------------------
+def check_gemv(pw, ref, x, y_dtype=q.OUT_F32):
+    t = x.shape[0]
+    y = torch.empty(t, pw.n, dtype=torch.float32 if y_dtype == q.OUT_F32 else torch.bfloat16,
+                    device=DEV)
+    ws = q.Workspace(DEV).ensure(q.qlin_gemv_workspace_bytes(pw, t))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q.qlin_gemv(pw, x.to(DEV), y, y_dtype, workspace=ws, dev_status=status)
+    yr, br = oracle.gemv(ref, bits16(x), nthreads=8)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    got = y.float().cpu().numpy().astype(np.float64)
+    tol = 1e-3 * br
+    if y_dtype == q.OUT_BF16:
+        tol = tol + np.abs(yr) * 2.0 ** -8
+    bad = np.abs(got - yr) > tol
+    assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
+    return got, yr
+
+
+@pytest.mark.parametrize("fmt", list(FMTS))
+@pytest.mark.parametrize("t", [1, 3, 4, 5, 17, 33, 64])
+def test_gemv_small_shapes(fmt, t):
+    n, k = 200, 1216  # ragged rows; K not a multiple of the K-split
+    w = synth.weights_f32(n, k, seed=200 + t)
+    x = synth.activations_bf16(t, k, seed=300 + t)
+    ref = oracle.pack(FMTS[fmt], w.numpy())
+    pw = pack_gpu(FMTS[fmt], w.to(DEV))
+    check_gemv(pw, ref, x, q.OUT_F32)
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q5", "fp8"])
+def test_gemv_bf16_output_and_long_k(fmt):
+    n, k, t = 96, 17408, 2
+    w = synth.weights_f32(n, k, seed=5)
+    x = synth.activations_bf16(t, k, seed=6)
+    ref = oracle.pack(FMTS[fmt], w.numpy())
+    pw = pack_gpu(FMTS[fmt], w.to(DEV))
+    check_gemv(pw, ref, x, q.OUT_BF16)
+
+
+def test_gemv_bf16_weights_prefill_sizes():
+    # GDN a/b projection kept in BF16: 96 x 5120 at a prefill chunk
+    n, k, t = 96, 5120, 512
+    w = synth.weights_f32(n, k, seed=9)
+    x = synth.activations_bf16(t, k, seed=10)
+    ref = oracle.pack(q.BF16, w.numpy())
+    pw = pack_gpu(q.BF16, w.to(DEV))
+    check_gemv(pw, ref, x, q.OUT_F32)
+
+
+@pytest.mark.parametrize("name,fmt,n,k,t", [
+    ("gate_up_q4", q.Q4_G64, 34816, 5120, 4),
+    ("down_q5", q.Q5_G64, 5120, 17408, 33),
+    ("q8_5120", q.Q8_G32, 5120, 5120, 17),
+    ("head_fp8", q.FP8_ROW, 152064, 5120, 1),
+])
+def test_gemv_full_size_sampled_rows(name, fmt, n, k, t):
+    """Full-size weights in the bench's launch configuration; the oracle
+    checks a sample of rows (packing is row-independent)."""
+    w = synth.weights_f32(n, k, seed=synth.seed_for(1, 0), device=DEV)
+    x = synth.activations_bf16(t, k, seed=synth.seed_for(1, 1), device=DEV)
+    pw = pack_gpu(fmt, w)
+    y = torch.empty(t, n, dtype=torch.float32, device=DEV)
+    ws = q.Workspace(DEV).ensure(q.qlin_gemv_workspace_bytes(pw, t))
+    q.qlin_gemv(pw, x, y, q.OUT_F32, workspace=ws)
+    g = torch.Generator().manual_seed(1)
+    rows = torch.cat([torch.randperm(n, generator=g)[:61], torch.tensor([0, n - 1])])
+    ref = oracle.pack(fmt, w[rows.to(DEV)].cpu().numpy())
+    got_packed = {"codes": None}
+    yr, br = oracle.gemv(ref, bits16(x), nthreads=8)
+    torch.cuda.synchronize()
+    got = y[:, rows.to(DEV)].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - yr) <= 1e-3 * br)
+    # packed rows bit-exact as well
+    sub = gpu_packed_to_numpy(pw)
+    for key in ("codes", "hibits", "scales"):
+        if ref[key] is not None:
+            assert np.array_equal(sub[key][rows.numpy()], ref[key]), key
+    del got_packed
+
+
+# ---------------------------------------------------------------------------
+# int8 route
+# ---------------------------------------------------------------------------
+def run_gemm_a8(pw, x, fused=True, debug=True, y_dtype=q.OUT_F32):
+    t, k = x.shape
+    n = pw.n
+    xd = x.to(DEV)
+    y = torch.empty(t, n, dtype=torch.float32 if y_dtype == q.OUT_F32 else torch.bfloat16, device=DEV)
+    dbg = torch.zeros(t, n, k // 64, dtype=torch.int32, device=DEV) if debug else None
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    flags = q.DEBUG_GROUP_SUMS if debug else 0
+    if fused:
+        ws = q.Workspace(DEV).ensure(q.qlin_gemm_a8_workspace_bytes(t, n, k))
+        q.qlin_gemm_a8(pw, y, x=xd, y_dtype=y_dtype, flags=flags, sums_dbg=dbg, workspace=ws,
+                       dev_status=status)
+    else:
+        xq = torch.empty(t, k, dtype=torch.int8, device=DEV)
+        xs = torch.empty(t, k // 64, dtype=torch.float32, device=DEV)
+        q.qlin_quantize_act(xd, xq, xs)
+        q.qlin_gemm_a8(pw, y, xq=xq, xs=xs, y_dtype=y_dtype, flags=flags, sums_dbg=dbg,
+                       dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return y, dbg
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q5"])
+@pytest.mark.parametrize("n,k,t", [(128, 256, 128), (256, 512, 130), (200, 640, 257), (384, 1152, 1),
+                                   (128, 5120, 64)])
+def test_gemm_a8_group_sums_bit_exact_and_output(fmt, n, k, t):
+    w = synth.weights_f32(n, k, seed=400 + n + k)
+    x = synth.activations_bf16(t, k, seed=500 + t)
+    ref = oracle.pack(FMTS[fmt], w.numpy())
+    pw = pack_gpu(FMTS[fmt], w.to(DEV), allow_a8=True)
+    y, dbg = run_gemm_a8(pw, x, fused=True, debug=True)
+    qa, as_ = oracle.quantize_act(bits16(x))
+    S = oracle.group_sums(ref, qa)
+    assert np.array_equal(dbg.cpu().numpy(), S)
+    yr, br = oracle.gemm_a8(ref, qa, as_, nthreads=8)
+    got = y.cpu().numpy().astype(np.float64)
+    bad = np.abs(got - yr) > 5e-6 * br
+    assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
+
+
+@pytest.mark.parametrize("fmt", ["q4", "q5"])
+def test_gemm_a8_prequantized_and_bf16_out(fmt):
+    n, k, t = 256, 1024, 300
+    w = synth.weights_f32(n, k, seed=41)
+    x = synth.activations_bf16(t, k, seed=42)
+    ref = oracle.pack(FMTS[fmt], w.numpy())
+    pw = pack_gpu(FMTS[fmt], w.to(DEV), allow_a8=True)
+    y, _ = run_gemm_a8(pw, x, fused=False, debug=False, y_dtype=q.OUT_BF16)
+    qa, as_ = oracle.quantize_act(bits16(x))
+    yr, br = oracle.gemm_a8(ref, qa, as_, nthreads=8)
+    got = y.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - yr) <= 5e-6 * br + np.abs(yr) * 2.0 ** -8)
+
+
+def test_gemm_a8_extreme_codes():
+    """All codes at their extremes: |S| = 64 * 15 * 127 per group, exact."""
+    n, k, t = 128, 512, 128
+    w = torch.full((n, k), 0.5, dtype=torch.float32)
+    w[::2] *= -1
+    x = torch.full((t, k), 2.0, dtype=torch.float32).to(torch.bfloat16)
+    pw = pack_gpu(q.Q5_G64, w.to(DEV), allow_a8=True)
+    y, dbg = run_gemm_a8(pw, x, fused=True, debug=True)
+    S = dbg.cpu().numpy()
+    assert np.all(np.abs(S) == 64 * 15 * 127)
+    ref = oracle.pack(q.Q5_G64, w.numpy())
+    qa, as_ = oracle.quantize_act(bits16(x))
+    assert np.array_equal(S, oracle.group_sums(ref, qa))
+
+
+@pytest.mark.parametrize("name,fmt,n,k", [("gate_up_q4", q.Q4_G64, 34816, 5120),
+                                          ("down_q5", q.Q5_G64, 5120, 17408)])
+def test_gemm_a8_full_size_sampled(name, fmt, n, k):
+    t = 2048
+    w = synth.weights_f32(n, k, seed=synth.seed_for(3, 0), device=DEV)
+    x = synth.activations_bf16(t, k, seed=synth.seed_for(3, 1), device=DEV)
+    pw = pack_gpu(fmt, w, allow_a8=True)
+    y = torch.empty(t, n, dtype=torch.float32, device=DEV)
+    ws = q.Workspace(DEV).ensure(q.qlin_gemm_a8_workspace_bytes(t, n, k))
+    q.qlin_gemm_a8(pw, y, x=x, y_dtype=q.OUT_F32, workspace=ws)
+    g = torch.Generator().manual_seed(3)
+    rows = torch.randperm(n, generator=g)[:24]
+    toks = torch.cat([torch.randperm(t, generator=g)[:14], torch.tensor([0, t - 1])])
+    ref = oracle.pack(fmt, w[rows.to(DEV)].cpu().numpy())
+    qa, as_ = oracle.quantize_act(bits16(x[toks.to(DEV)]))
+    yr, br = oracle.gemm_a8(ref, qa, as_, nthreads=8)
+    torch.cuda.synchronize()
+    got = y[toks.to(DEV)][:, rows.to(DEV)].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - yr) <= 5e-6 * br)
