@@ -45,6 +45,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
+    p.add_argument("--case", default=None,
+                   help="run one kernel case only (for profilers): gemv:<q4|q5|q8|fp8|bf16>:<N>x<K>:T<t> "
+                        "or gemm_a8:<q4|q5>:<N>x<K>:T<t> or quantize:<T>x<K> or decode:<R>x<C>")
     return p.parse_args()
 
 
@@ -108,8 +111,11 @@ class Clocks:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index = index
+    def __init__(self, device_index):
+        try:
+            self.index = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.index = str(device_index)
         self.proc = None
         self.path = None
 
@@ -120,7 +126,7 @@ class Clocks:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -240,11 +246,19 @@ def run_ours(args, dist):
                 else:
                     f()
 
+    clocks = Clocks(dist.local)
+    clocks.start()  # sampling covers the warm-up (at least ~1 s of this load) and the timed region
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    clocks = Clocks(dist.local)
-    clocks.start()
+    t_settle = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_settle < 1.0:
+        step(i)
+        i += 1
+        if i % 50 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -510,8 +524,58 @@ def cpu_baseline(target_s):
                       f"{reps} repetitions ({dt:.1f} s), rows split over {cores} threads"}
 
 
+
+def run_case(args):
+    """One kernel case, W warm-up + K timed calls; prints a short JSON line."""
+    import quantized_weight_linear_qlin_b200 as q
+    import synth
+    from quantized_weight_linear_qlin_b200 import _build
+    _build.build()
+    dev = torch.device("cuda", 0)
+    fmts = {"q4": q.Q4_G64, "q5": q.Q5_G64, "q8": q.Q8_G32, "fp8": q.FP8_ROW, "bf16": q.BF16}
+    parts = args.case.split(":")
+    kind = parts[0]
+    ws = q.Workspace(dev)
+    if kind in ("gemv", "gemm_a8"):
+        fmt = fmts[parts[1]]
+        n, k = (int(v) for v in parts[2].split("x"))
+        t = int(parts[3][1:])
+        pw = packed(q, synth, fmt, n, k, 1, dev, allow_a8=kind == "gemm_a8")
+        x = synth.activations_bf16(t, k, seed=2, device=dev)
+        y = torch.empty(t, n, dtype=torch.bfloat16, device=dev)
+        if kind == "gemv":
+            ws.ensure(q.qlin_gemv_workspace_bytes(pw, t))
+            fn = lambda: q.qlin_gemv(pw, x, y, q.OUT_BF16, workspace=ws)  # noqa: E731
+            units, unit = gemv_bytes(pw, t), "GB/s"
+        else:
+            ws.ensure(q.qlin_gemm_a8_workspace_bytes(t, n, k))
+            fn = lambda: q.qlin_gemm_a8(pw, y, x=x, workspace=ws)  # noqa: E731
+            units, unit = 2 * t * n * k, "TOPS"
+    elif kind == "quantize":
+        t, k = (int(v) for v in parts[1].split("x"))
+        x = synth.activations_bf16(t, k, seed=2, device=dev)
+        xq = torch.empty(t, k, dtype=torch.int8, device=dev)
+        xs = torch.empty(t, k // 64, dtype=torch.float32, device=dev)
+        fn = lambda: q.qlin_quantize_act(x, xq, xs)  # noqa: E731
+        units, unit = t * k * 2 + t * k + t * (k // 64) * 4, "GB/s"
+    elif kind == "decode":
+        r, c = (int(v) for v in parts[1].split("x"))
+        words, sc = synth.mxfp8_source(r, c, seed=2, device=dev)
+        out = torch.empty(r, c, dtype=torch.int16, device=dev)
+        fn = lambda: q.qlin_decode_mxfp8(words, sc, r, c, out)  # noqa: E731
+        units, unit = r * c + r * (c // 32) + 2 * r * c, "GB/s"
+    else:
+        raise SystemExit(f"unknown case {args.case}")
+    ms = time_fn(fn, iters=args.steps, warm=args.warmup)
+    per_ms = 1e6 if unit == "GB/s" else 1e9
+    print(json.dumps({"case": args.case, "ms": round(ms, 5), unit: round(units / ms / per_ms, 2)}))
+
+
 def main():
     args = parse()
+    if args.case:
+        run_case(args)
+        return
     dist = Dist(args.gpus)
     if args.impl == "reference":
         if dist.rank != 0:

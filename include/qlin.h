@@ -185,7 +185,8 @@ QLIN_API int qlin_gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, size_
 
 /* Int8-route projection (prefill).  Weights must be Q4_G64 or Q5_G64
  * (QLIN_ERR_UNSUPPORTED otherwise) carrying QLIN_ALLOW_A8
- * (QLIN_ERR_NOT_PERMITTED otherwise).  Activations either as x_bf16 (the
+ * (QLIN_ERR_NOT_PERMITTED otherwise) and K % 128 == 0 (QLIN_ERR_UNSUPPORTED
+ * otherwise).  Activations either as x_bf16 (the
  * per-token per-64 quantizer runs inside the call, xq/xs must be NULL) or
  * pre-quantized as xq int8[T][K] + xs float32[T][K/64] (x_bf16 NULL).
  * S[t][n][g] = sum over the group of xq * q (int32, exact);

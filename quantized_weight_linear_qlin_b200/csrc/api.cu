@@ -11,6 +11,10 @@ namespace qlin {
 size_t gemv_cc_workspace_bytes(const qlin_weights& w, int64_t t);
 int launch_gemv_cc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                    const Exec& ex, float* acc_ws);
+bool gemv_tc_supported(const qlin_weights& w, int64_t t);
+size_t gemv_tc_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
+int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
+                   const Exec& ex);
 
 namespace {
 
@@ -98,13 +102,17 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
   return r == CUDA_SUCCESS ? QLIN_OK : QLIN_ERR_CUDA;
 }
 
+// T <= 64 runs on the tensor cores; BF16 weights at prefill sizes (T > 64)
+// and Q5 rows whose high-bit plane is not 16-byte aligned per row use the
+// CUDA-core kernel.
 size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
-  (void)num_sms;
+  if (gemv_tc_supported(w, t)) return gemv_tc_workspace_bytes(w, t, num_sms);
   return gemv_cc_workspace_bytes(w, t);
 }
 
 int launch_gemv(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                 const Exec& ex) {
+  if (gemv_tc_supported(w, t)) return launch_gemv_tc(w, x, t, y, y_dtype, ex);
   return launch_gemv_cc(w, x, t, y, y_dtype, ex, (float*)ex.workspace);
 }
 
@@ -213,7 +221,7 @@ int qlin_gemm_a8(const qlin_weights* w, const uint16_t* x_bf16, const int8_t* xq
   if (rc) return rc;
   if (w->fmt != QLIN_Q4_G64 && w->fmt != QLIN_Q5_G64) return QLIN_ERR_UNSUPPORTED;
   if (!(w->flags & QLIN_ALLOW_A8)) return QLIN_ERR_NOT_PERMITTED;
-  if (w->fmt == QLIN_Q5_G64 && w->k % 128) return QLIN_ERR_UNSUPPORTED;
+  if (w->k % 128) return QLIN_ERR_UNSUPPORTED;
   if (t <= 0 || !y || !aligned16(y)) return QLIN_ERR_INVALID_ARG;
   if (y_dtype != QLIN_OUT_BF16 && y_dtype != QLIN_OUT_F32) return QLIN_ERR_INVALID_ARG;
   const bool fused = x_bf16 != nullptr;

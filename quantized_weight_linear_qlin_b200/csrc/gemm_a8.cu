@@ -84,11 +84,12 @@ struct __align__(1024) StageSmem {
   uint8_t b[2][BN * 128];        // int8 activations, two atoms
   uint8_t raw[BM * 128];         // packed nibbles of 256 columns (swizzled)
   uint8_t hib[BM * 32];          // Q5 high bits of 256 columns
+  float xsb[GPS * BN];           // activation scales of the stage, [group][token]
+  __half wsb[BM * GPS];          // weight scales of the stage, [row][group]
 };
 
 struct Smem {
   StageSmem st[STAGES];
-  float xsb[2][GPS * BN];        // activation scales of a stage, [group][token]
   uint64_t full[STAGES], a_ready[STAGES], empty[STAGES];
   uint64_t d_full[2], d_empty[2], drain;
   uint32_t tmem_base;
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.full[s], 1 + 32);  // TMA issue + 32 scale-copy arrivals
       mbar_init(&sm.a_ready[s], NUM_UNPACK_THREADS);
       mbar_init(&sm.empty[s], 1 + NUM_EPI_WARPS * 32);
     }
@@ -177,27 +178,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = sm.tmem_base;
 
   if (warp == WARP_TMA) {
-    if (lane == 0) {
-      // activations come from the quantizer kernel launched just before
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      int64_t issued = 0;
-      for (int64_t kc = 0; kc < nchunks; ++kc) {
-        const int s = (int)(kc % STAGES);
-        const uint32_t par = (uint32_t)((kc / STAGES) & 1);
-        if (aborted(sm)) break;
-        if (!mbar_wait(&sm.empty[s], par ^ 1)) { set_abort(sm, args.dev_status); break; }
+    // lane 0 issues the TMA copies; all 32 lanes copy the stage's weight and
+    // activation scales into shared memory with cp.async (same barrier).
+    // The activations come from the quantizer kernel launched just before.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    int64_t issued = 0;
+    for (int64_t kc = 0; kc < nchunks; ++kc) {
+      const int s = (int)(kc % STAGES);
+      const uint32_t par = (uint32_t)((kc / STAGES) & 1);
+      if (!__all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.empty[s], par ^ 1))) {
+        if (lane == 0) set_abort(sm, args.dev_status);
+        break;
+      }
+      const int gcount = (int)min((int64_t)GPS, ng - kc * GPS);
+      if (lane == 0) {
         uint32_t bytes = BM * 128 + 2 * BN * 128 + (BITS == 5 ? BM * 32 : 0);
         mbar_arrive_expect_tx(&sm.full[s], bytes);
         tma_load_2d(sm.st[s].raw, &tm_codes, &sm.full[s], (int)(kc * 128), (int)n0);
         if (BITS == 5) tma_load_2d(sm.st[s].hib, &tm_hib, &sm.full[s], (int)(kc * 32), (int)n0);
         tma_load_2d(sm.st[s].b[0], &tm_act, &sm.full[s], (int)(kc * BKC), (int)t0);
         tma_load_2d(sm.st[s].b[1], &tm_act, &sm.full[s], (int)(kc * BKC + 128), (int)t0);
-        ++issued;
       }
-      // let every copy in flight land before the CTA can leave
+      // weight scales: two groups (4 bytes) per copy; K % 128 == 0 keeps them aligned
+      for (int rr = lane; rr < BM; rr += 32) {
+        const int64_t grow = n0 + rr;
+        if (grow < args.n)
+          for (int gp = 0; gp < gcount; gp += 2)
+            cp_async_4(&sm.st[s].wsb[rr * GPS + gp], args.ws + grow * ng + kc * GPS + gp);
+      }
+      // activation scales, [group][token]
+      for (int tt = lane; tt < BN; tt += 32) {
+        const int64_t gt = t0 + tt;
+        if (gt < args.t)
+          for (int gi = 0; gi < gcount; ++gi)
+            cp_async_4(&sm.st[s].xsb[gi * BN + tt], args.xs + gt * ng + kc * GPS + gi);
+      }
+      cp_async_arrive_noinc(&sm.full[s]);
+      ++issued;
+    }
+    // let every copy in flight land before the CTA can leave
+    if (lane == 0)
       for (int64_t kc = issued > STAGES ? issued - STAGES : 0; kc < issued; ++kc)
         mbar_wait(&sm.full[kc % STAGES], (uint32_t)((kc / STAGES) & 1));
-    }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
       const uint32_t idesc = idesc_i8(BM, BN);
@@ -276,32 +298,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = quarter * 32 + lane;
     const int64_t grow = n0 + row;
     const int col0 = half * 64;
-    const int et = threadIdx.x;  // 0..255
     float acc[64];
 #pragma unroll
     for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
     int64_t G = 0;
-    // Every epilogue thread runs every chunk (the named barrier below needs all
-    // 256); after an abort the waits are skipped instead of the loop.
     for (int64_t kc = 0; kc < nchunks; ++kc) {
       const int s = (int)(kc % STAGES);
       const int gcount = (int)min((int64_t)GPS, ng - kc * GPS);
-      // stage the activation scales of this chunk: [group][token]
-      float* xsb = sm.xsb[kc & 1];
-      for (int i = et; i < BN * GPS; i += NUM_EPI_WARPS * 32) {
-        const int gi = i / BN, tt = i % BN;
-        const int64_t gt = t0 + tt, gg = kc * GPS + gi;
-        xsb[i] = (gt < args.t && gi < gcount) ? args.xs[gt * ng + gg] : 0.0f;
+      // acquire the stage (its scale copies landed when the barrier completed)
+      if (__any_sync(0xffffffffu, aborted(sm)) ||
+          !__all_sync(0xffffffffu, mbar_wait(&sm.full[s], (uint32_t)((kc / STAGES) & 1)))) {
+        set_abort(sm, args.dev_status);
+        break;
       }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float* xsb = sm.st[s].xsb;
+      const uint2 wsr = *(const uint2*)(&sm.st[s].wsb[row * GPS]);
+      const float ws0 = __low2float(*(const __half2*)&wsr.x), ws1 = __high2float(*(const __half2*)&wsr.x);
+      const float ws2 = __low2float(*(const __half2*)&wsr.y), ws3 = __high2float(*(const __half2*)&wsr.y);
+      bool ok = true;
       for (int gi = 0; gi < gcount; ++gi, ++G) {
         const int b = (int)(G & 1);
-        // warp-uniform decisions: tcgen05.ld below needs the whole warp
-        if (__any_sync(0xffffffffu, aborted(sm))) continue;
-        const float wsc = grow < args.n ? __half2float(args.ws[grow * ng + kc * GPS + gi]) : 0.0f;
+        const float wsc = gi == 0 ? ws0 : gi == 1 ? ws1 : gi == 2 ? ws2 : ws3;
+        // warp-uniform: tcgen05.ld below needs the whole warp
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.d_full[b], (uint32_t)((G >> 1) & 1)))) {
-          set_abort(sm, args.dev_status);
-          continue;
+          ok = false;
+          break;
         }
         tc_fence_after();
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + b * BN + col0;
@@ -333,7 +354,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!aborted(sm)) mbar_arrive(&sm.empty[s]);
+      if (!ok) {
+        set_abort(sm, args.dev_status);
+        break;
+      }
+      mbar_arrive(&sm.empty[s]);
     }
     if (!__any_sync(0xffffffffu, aborted(sm)) && grow < args.n) {
       const int64_t base = (t0 + col0) * args.n + grow;
