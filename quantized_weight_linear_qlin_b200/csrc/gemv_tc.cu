@@ -6,23 +6,29 @@
 //
 // Why tensor cores for a bandwidth-bound GEMV: at T >= 2 the CUDA cores cannot
 // both unpack the codes and do T FMAs per weight at HBM speed.  Here the CUDA
-// cores only unpack; the tcgen05 MMA does the dot products.
+// cores only unpack; tcgen05 MMAs do the dot products.
 //
-// One persistent CTA per SM walks a contiguous range of (128-row tile, K-chunk)
-// units (stream-K), so every SM streams the same number of weight bytes:
-//   warp 0      TMA: 128 rows x 128 bytes of packed codes (+ the Q5 high-bit
-//               plane) and the matching activation columns, into a ring of
-//               shared-memory stages;
-//   warps 4-7   dequantize: thread r owns weight row r; it expands one group's
-//               codes to exact BF16 integers (exponent-bias tricks, no
-//               conversions) and writes them with tcgen05.st as the MMA's A
-//               operand straight into tensor memory (lane r);
-//   warp 1      issues tcgen05.mma.kind::f16 (A from tensor memory, B = the
-//               activations from shared memory, M = 128, N = T padded to 16)
-//               into a fresh FP32 accumulator per quantization group;
-//   warps 8-11  epilogue: tcgen05.ld each group's 128 x T sums and apply the
-//               group's FP16 scale in FP32 registers (row-scaled FP8 and BF16
-//               weights accumulate a whole tile segment in the tensor core).
+// One persistent CTA per SM walks a contiguous range of units (a unit is one
+// 128-row tile x 256 bytes of packed codes per row, or 128 bytes when the
+// activation tile would not leave room for three stages), so every SM streams
+// the same number of weight bytes (stream-K):
+//   warp 0      TMA: the unit's packed codes (two 128-byte-wide boxes: wide
+//               row segments keep HBM efficient), the Q5 high-bit plane and the
+//               matching activation columns into a ring of shared-memory
+//               stages; its 32 lanes cp.async the group scales;
+//   warpgroups 1-2  take turns on batches of quantization groups: every thread
+//               owns one weight row, expands the batch's codes to exact BF16
+//               integers (exponent-bias tricks, no conversions) and writes them
+//               with tcgen05.st as the MMA's A operand straight into tensor
+//               memory; after a warpgroup barrier one elected thread issues the
+//               batch's tcgen05.mma.kind::f16 (A in tensor memory, B = the
+//               activations in shared memory, M = 128, N = T padded to 16), one
+//               FP32 accumulator per group, and commits once.  Two issuing
+//               threads: one thread issues an MMA only every ~65 cycles;
+//   warpgroup 3 the epilogue reads a batch's 128 x T sums with tcgen05.ld,
+//               applies each group's FP16 scale in FP32 registers and re-zeroes
+//               the accumulators (every MMA accumulates: one that overwrites its
+//               accumulator costs about four that accumulate).
 // Tiles split between two CTAs meet in a workspace; the last CTA to arrive
 // sums the parts in a fixed order (deterministic) and writes y.
 #include "qlin_internal.cuh"
@@ -30,53 +36,76 @@
 namespace qlin {
 namespace {
 
-constexpr int TC_THREADS = 16 * 32;
-constexpr int W_TMA = 0, W_MMA = 1, W_DQ0 = 4, W_EPI0 = 8, W_DQB0 = 12;
-constexpr int NA = 4;  // A stages in tensor memory
-constexpr int ND = 4;  // accumulator stages in tensor memory
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int CODES_BYTES = 128 * 128;
+constexpr int BOX_BYTES = 128 * 128;  // one TMA box of codes: 128 rows x 128 bytes
 constexpr int SMEM_BUDGET = 212992;
+constexpr int NWG = 2;                // dequantizing / MMA-issuing warpgroups
+constexpr int THREADS = 16 * 32;      // control, 2 x dequant, epilogue warpgroups
+constexpr int W_DQ0 = 4, W_EPI0 = 12;
 
+// Per format: K per quantization group, groups per 128-byte box of codes,
+// high-bit plane, per-group scales.
 template <int FMT>
 struct TcT;
 template <>
 struct TcT<QLIN_Q4_G64> {
-  static constexpr int KC = 256, GK = 64, GPC = 4, BOXES = 4;
+  static constexpr int GK = 64, GPB = 4;
   static constexpr bool PER_GROUP = true, HIB = false;
 };
 template <>
 struct TcT<QLIN_Q5_G64> {
-  static constexpr int KC = 256, GK = 64, GPC = 4, BOXES = 4;
+  static constexpr int GK = 64, GPB = 4;
   static constexpr bool PER_GROUP = true, HIB = true;
 };
 template <>
 struct TcT<QLIN_Q8_G32> {
-  static constexpr int KC = 128, GK = 32, GPC = 4, BOXES = 2;
+  static constexpr int GK = 32, GPB = 4;
   static constexpr bool PER_GROUP = true, HIB = false;
 };
 template <>
 struct TcT<QLIN_FP8_ROW> {
-  static constexpr int KC = 128, GK = 64, GPC = 2, BOXES = 2;
-  static constexpr bool PER_GROUP = false, HIB = false;
+  static constexpr int GK = 64, GPB = 2;
+  static constexpr bool PER_GROUP = false, HIB = false;  // one scale per row, applied at the end
 };
 template <>
 struct TcT<QLIN_BF16> {
-  static constexpr int KC = 64, GK = 64, GPC = 1, BOXES = 1;
+  static constexpr int GK = 64, GPB = 1;
   static constexpr bool PER_GROUP = false, HIB = false;
+};
+
+template <int FMT, int TP, int UB>
+struct Layout {
+  using Tr = TcT<FMT>;
+  static constexpr int GPC = Tr::GPB * UB;            // groups per unit
+  static constexpr int KC = Tr::GK * GPC;             // K columns per unit
+  static constexpr int XBOXES = KC / 64;              // activation boxes (64 columns each)
+  static constexpr int X_BYTES = XBOXES * TP * 128;
+  static constexpr int HIB_BYTES = Tr::HIB ? UB * 128 * 32 : 0;
+  static constexpr int SC_ROW = Tr::PER_GROUP ? GPC * 2 : 0;  // scale bytes per row per unit
+  static constexpr int SC_BYTES = 128 * SC_ROW;
+  static constexpr int TMA_BYTES = UB * BOX_BYTES + X_BYTES + HIB_BYTES;
+  static constexpr int STAGE = TMA_BYTES + SC_BYTES;
+  static constexpr int NS = (SMEM_BUDGET / STAGE) > 8 ? 8 : (SMEM_BUDGET / STAGE);
 };
 
 template <int FMT, int TP>
 struct Cfg {
   using Tr = TcT<FMT>;
-  static constexpr int X_BYTES = Tr::BOXES * TP * 128;
-  static constexpr int HIB_BYTES = Tr::HIB ? 128 * 32 : 0;
-  static constexpr int SC_BYTES = Tr::PER_GROUP ? 128 * Tr::GPC * 2 : 0;  // 8 B of scales per row
-  static constexpr int TMA_BYTES = CODES_BYTES + X_BYTES + HIB_BYTES;
-  static constexpr int STAGE = TMA_BYTES + SC_BYTES;
-  static constexpr int NS = (SMEM_BUDGET / STAGE) > 8 ? 8 : (SMEM_BUDGET / STAGE);
-  static constexpr int ACOLS = Tr::GK / 2;  // tensor-memory columns of one A stage
-  static constexpr size_t SMEM = (size_t)NS * STAGE + 1024 + 512;
+  // two 128-byte boxes per unit when three stages still fit, else one
+  static constexpr int UB = Layout<FMT, TP, 2>::NS >= 3 ? 2 : 1;
+  using L = Layout<FMT, TP, UB>;
+  static constexpr int GPC = L::GPC, KC = L::KC, NS = L::NS;
+  static constexpr int ACOLS = Tr::GK / 2;            // tensor-memory columns of one group's A
+  static constexpr bool fits(int gb) { return NWG * (gb * ACOLS + 2 * gb * TP) <= (int)TMEM_COLS; }
+  // groups per batch: one barrier, one commit and one epilogue wait per batch
+  static constexpr int GB = (GPC % 4 == 0 && fits(4)) ? 4 : (GPC % 2 == 0 && fits(2)) ? 2 : 1;
+  static constexpr int BPU = GPC / GB;                // batches per unit
+  static constexpr int A_COLS = GB * ACOLS;           // a warpgroup's A slot
+  static constexpr int D_COLS = GB * TP;              // one accumulator slot (a batch)
+  static constexpr int WG_COLS = A_COLS + 2 * D_COLS; // per warpgroup: A slot + two accumulator slots
+  static_assert(NS >= 2, "pipeline needs two stages");
+  static_assert(NWG * WG_COLS <= (int)TMEM_COLS, "tensor memory budget");
+  static constexpr size_t SMEM = (size_t)NS * L::STAGE + 1024 + 512;
 };
 
 struct TcArgs {
@@ -86,7 +115,7 @@ struct TcArgs {
   int* counters;    // [tiles]
   int32_t* dev_status;
   int64_t n, k, t;
-  int64_t cpt;      // K-chunks per tile
+  int64_t cpt;      // units per tile
   int64_t units;    // tiles * cpt
   int y_dtype;
 };
@@ -187,28 +216,38 @@ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t U, int64_t P) {
   return i;
 }
 
+// A ring position: slot index and the parity of its current use.  Advancing
+// by one avoids integer division in the loops (64-bit divisions are slow).
+struct Ring {
+  int slot, phase;
+  __device__ __forceinline__ void next(int n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1;
+    }
+  }
+};
+
 template <int FMT, int TP>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                    const __grid_constant__ CUtensorMap tm_hib,
                    const __grid_constant__ CUtensorMap tm_x, TcArgs args) {
   using Tr = TcT<FMT>;
   using C = Cfg<FMT, TP>;
-  constexpr int NS = C::NS;
+  using L = typename C::L;
+  constexpr int NS = C::NS, UB = C::UB, GPC = C::GPC, GB = C::GB, BPU = C::BPU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* codes_s = base;
-  uint8_t* x_s = codes_s + NS * CODES_BYTES;
-  uint8_t* hib_s = x_s + NS * C::X_BYTES;
-  uint8_t* sc_s = hib_s + NS * C::HIB_BYTES;
-  uint64_t* full = (uint64_t*)(sc_s + NS * C::SC_BYTES);
+  uint8_t* codes_s = base;                                  // NS x UB boxes
+  uint8_t* x_s = codes_s + NS * UB * BOX_BYTES;             // NS x X_BYTES
+  uint8_t* hib_s = x_s + NS * L::X_BYTES;                   // NS x HIB_BYTES
+  uint8_t* sc_s = hib_s + NS * L::HIB_BYTES;                // NS x SC_BYTES
+  uint64_t* full = (uint64_t*)(sc_s + NS * L::SC_BYTES);
   uint64_t* empty = full + NS;
-  uint64_t* a_full = empty + NS;
-  uint64_t* a_empty = a_full + NA;
-  uint64_t* d_full = a_empty + NA;
-  uint64_t* d_empty = d_full + ND;
-  uint64_t* drain = d_empty + ND;
-  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  uint64_t* d_full = empty + NS;        // [NWG][2]
+  uint64_t* d_empty = d_full + 2 * NWG; // [NWG][2]
+  uint32_t* tmem_slot = (uint32_t*)(d_empty + 2 * NWG);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   volatile int* fix_slot = (volatile int*)(tmem_slot + 2);
 
@@ -218,29 +257,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int64_t u0 = unit_start(blockIdx.x, U, P), u1 = unit_start(blockIdx.x + 1, U, P);
   const int64_t ng = args.k / Tr::GK;  // groups per row
   const int T = (int)args.t;
+  const int cpt = (int)args.cpt;
+  const int nunits = (int)(u1 - u0);
+  const int tile0 = (int)(u0 / cpt), ch0 = (int)(u0 % cpt);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1 + 32);             // TMA issue + 32 scale-copy arrivals
-      mbar_init(&empty[s], 1 + 2 * 128 + 128);  // MMA commit + both dequant groups + epilogue
+      mbar_init(&full[s], 1 + 32);  // TMA issue + 32 scale-copy arrivals
+      mbar_init(&empty[s], 1);      // released by the epilogue once the unit is done
     }
-    for (int a = 0; a < NA; ++a) {
-      mbar_init(&a_full[a], 128);
-      mbar_init(&a_empty[a], 1);
+    for (int i = 0; i < 2 * NWG; ++i) {
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_empty[i], 128);
     }
-    for (int d = 0; d < ND; ++d) {
-      mbar_init(&d_full[d], 1);
-      mbar_init(&d_empty[d], 128);
-    }
-    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == W_MMA) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == W_TMA && lane == 0) {
+  if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_codes);
     tma_prefetch_desc(&tm_x);
     if (Tr::HIB) tma_prefetch_desc(&tm_hib);
@@ -249,132 +286,157 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_a = tmem;
-  const uint32_t tmem_d = tmem + NA * C::ACOLS;
+  // warpgroup w: A slot at w * WG_COLS, accumulator slots j at + A_COLS + j * D_COLS
+  if (warp >= W_EPI0) {  // accumulators start at zero; the epilogue re-zeroes each after use
+    const uint32_t lo = (uint32_t)((warp & 3) * 32) << 16;
+#pragma unroll 1
+    for (int w = 0; w < NWG; ++w)
+#pragma unroll 1
+      for (int c = 0; c < 2 * C::D_COLS; c += 16)
+        tmem_fill_x16(tmem + lo + w * C::WG_COLS + C::A_COLS + c, 0u);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   auto abort_now = [&]() {
     *abort_flag = 1;
     report_timeout(args.dev_status);
   };
 
-  if (warp == W_TMA) {
-    // lane 0 issues the TMA copies; all 32 lanes copy the stage's group scales
-    // (8 bytes per row) with cp.async, tracked by the same barrier.
-    int64_t issued = 0;
-    for (int64_t u = u0; u < u1; ++u) {
-      const int64_t cu = u - u0;
-      const int s = (int)(cu % NS);
-      if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait(&empty[s], (uint32_t)(((cu / NS) & 1) ^ 1)))) {
+  if (warp == 0) {
+    // lane 0 issues the TMA copies; all 32 lanes copy the unit's group scales
+    // (SC_ROW bytes per row) with cp.async, tracked by the same barrier.
+    int issued = 0;
+    Ring ring{0, 0};
+    int tile = tile0, ch = ch0;
+    for (int cu = 0; cu < nunits; ++cu) {
+      const int s = ring.slot;
+      if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait(&empty[s], (uint32_t)(ring.phase ^ 1)))) {
         if (lane == 0) abort_now();
         break;
       }
-      const int64_t tile = u / args.cpt, ch = u % args.cpt;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], C::TMA_BYTES);
-        tma_load_2d(codes_s + s * CODES_BYTES, &tm_codes, &full[s], (int)(ch * 128), (int)(tile * 128));
-        if (Tr::HIB)
-          tma_load_2d(hib_s + s * C::HIB_BYTES, &tm_hib, &full[s], (int)(ch * 32), (int)(tile * 128));
+        mbar_arrive_expect_tx(&full[s], L::TMA_BYTES);
 #pragma unroll
-        for (int b = 0; b < Tr::BOXES; ++b)
-          tma_load_2d(x_s + s * C::X_BYTES + b * TP * 128, &tm_x, &full[s],
-                      (int)(ch * Tr::KC + b * 64), 0);
+        for (int b = 0; b < UB; ++b)
+          tma_load_2d(codes_s + (s * UB + b) * BOX_BYTES, &tm_codes, &full[s], (ch * UB + b) * 128, tile * 128);
+        if (Tr::HIB) tma_load_2d(hib_s + s * L::HIB_BYTES, &tm_hib, &full[s], ch * UB * 32, tile * 128);
+#pragma unroll
+        for (int b = 0; b < L::XBOXES; ++b)
+          tma_load_2d(x_s + s * L::X_BYTES + b * TP * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0);
       }
       if constexpr (Tr::PER_GROUP) {
-        const __half* src = (const __half*)args.scales + ch * Tr::GPC;
-        uint8_t* dst = sc_s + s * C::SC_BYTES;
+        const __half* src = (const __half*)args.scales + ch * GPC;
+        uint8_t* dst = sc_s + s * L::SC_BYTES;
 #pragma unroll
         for (int rr = lane; rr < 128; rr += 32) {
-          const int64_t row = tile * 128 + rr;
-          if (row < args.n) cp_async_8(dst + rr * 8, src + row * ng);
+          const int64_t row = (int64_t)tile * 128 + rr;
+          if (row < args.n) {
+            if constexpr (L::SC_ROW == 16) {
+              cp_async_8(dst + rr * 16, src + row * ng);
+              cp_async_8(dst + rr * 16 + 8, src + row * ng + 4);
+            } else {
+              cp_async_8(dst + rr * L::SC_ROW, src + row * ng);
+            }
+          }
         }
       }
       cp_async_arrive_noinc(&full[s]);
       ++issued;
+      ring.next(NS);
+      if (++ch == cpt) {
+        ch = 0;
+        ++tile;
+      }
     }
     if (lane == 0)
-      for (int64_t cu = issued > NS ? issued - NS : 0; cu < issued; ++cu)
+      for (int cu = issued > NS ? issued - NS : 0; cu < issued; ++cu)
         mbar_wait(&full[cu % NS], (uint32_t)((cu / NS) & 1));
-  } else if (warp == W_MMA) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, TP);
-      int64_t G = 0, D = 0;
-      for (int64_t u = u0; u < u1 && !*abort_flag; ++u) {
-        const int64_t cu = u - u0;
-        const int s = (int)(cu % NS);
-        if (!mbar_wait(&full[s], (uint32_t)((cu / NS) & 1))) { abort_now(); break; }
-        const int64_t ch = u % args.cpt;
-        const int gcount = (int)min((int64_t)Tr::GPC, ng - ch * Tr::GPC);
-        const bool seg_first = (u == u0) || ch == 0;
-        const bool seg_last = (u + 1 == u1) || ((u + 1) % args.cpt == 0);
-        const uint32_t xs_base = smem_u32(x_s + s * C::X_BYTES);
-        bool ok = true;
-        for (int gi = 0; gi < gcount; ++gi, ++G) {
-          const int a = (int)(G % NA);
-          const bool new_acc = Tr::PER_GROUP || (seg_first && gi == 0);
-          const bool close_acc = Tr::PER_GROUP || (seg_last && gi == gcount - 1);
-          const int d = (int)(D % ND);
-          if (!mbar_wait(&a_full[a], (uint32_t)((G / NA) & 1))) { ok = false; break; }
-          if (new_acc && !mbar_wait(&d_empty[d], (uint32_t)(((D / ND) & 1) ^ 1))) { ok = false; break; }
-          tc_fence_after();
-          const int kofs = gi * Tr::GK;  // K offset of the group inside the chunk
-          const uint32_t xaddr = xs_base + (kofs / 64) * TP * 128 + (kofs % 64) * 2;
-#pragma unroll
-          for (int kk = 0; kk < Tr::GK / 16; ++kk)
-            mma_f16_ts(tmem_d + d * TP, tmem_a + a * C::ACOLS + kk * 8, sdesc_k_sw128(xaddr + kk * 32),
-                       idesc, (kk > 0 || !new_acc) ? 1u : 0u);
-          tc_commit(&a_empty[a]);
-          if (close_acc) {
-            tc_commit(&d_full[d]);
-            ++D;
-          }
-        }
-        if (!ok) { abort_now(); break; }
-        tc_commit(&empty[s]);
-      }
-      tc_commit(drain);
-      mbar_wait(drain, 0);
-    }
-  } else if ((warp >= W_DQ0 && warp < W_DQ0 + 4) || warp >= W_DQB0) {
-    // two dequantizing warpgroups take alternate groups (A stages of matching parity)
-    const int wg = warp >= W_DQB0 ? 1 : 0;
+  } else if (warp >= W_DQ0 && warp < W_EPI0) {
+    // ---- dequantize + issue: warpgroup wg takes the batches b with b % NWG == wg
+    const int wg = (warp - W_DQ0) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_ofs = (uint32_t)(quarter * 32) << 16;
-    int64_t G = 0;
-    for (int64_t u = u0; u < u1; ++u) {
-      const int64_t cu = u - u0;
-      const int s = (int)(cu % NS);
-      if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait(&full[s], (uint32_t)((cu / NS) & 1)))) {
-        abort_now();
-        break;
-      }
-      const int64_t ch = u % args.cpt;
-      const int gcount = (int)min((int64_t)Tr::GPC, ng - ch * Tr::GPC);
-      const uint8_t* cs = codes_s + s * CODES_BYTES;
-      const uint8_t* hs = hib_s + s * C::HIB_BYTES;
-      bool ok = true;
-      for (int gi = 0; gi < gcount; ++gi, ++G) {
-        if ((int)(G & 1) != wg) continue;
-        uint32_t v[C::ACOLS];
-        dequant_group<FMT>(cs, hs, r, gi, v);
-        const int a = (int)(G % NA);
-        if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[a], (uint32_t)(((G / NA) & 1) ^ 1)))) {
-          ok = false;
-          break;
+    const bool issuer = quarter == 0 && lane == 0;
+    const uint32_t idesc = idesc_bf16(128, TP);
+    const uint32_t a_base = tmem + wg * C::WG_COLS;
+    const uint32_t d_base = a_base + C::A_COLS;
+    bool dead = false;  // after a timed-out wait: skip work, keep the barrier sequence
+    Ring ring{0, 0};
+    Ring dr{0, 0};       // this warpgroup's accumulator slot
+    int prev_slot = -1, prev_phase = 0;
+    int bw = 0;          // owner of the next batch
+    for (int cu = 0; cu < nunits; ++cu) {
+      const int s = ring.slot;
+      bool mine = false;
+      {
+        int w = bw;
+        for (int bi = 0; bi < BPU; ++bi) {
+          mine |= w == wg;
+          w = (w + 1 == NWG) ? 0 : w + 1;
         }
-        tc_fence_after();
-        if constexpr (C::ACOLS == 32)
-          tmem_st_x32(tmem_a + lane_ofs + a * C::ACOLS, v);
-        else
-          tmem_st_x16(tmem_a + lane_ofs + a * C::ACOLS, v);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&a_full[a]);
       }
-      if (!ok) { abort_now(); break; }
-      mbar_arrive(&empty[s]);
+      if (mine && !dead &&
+          !__all_sync(0xffffffffu, !*abort_flag && mbar_wait(&full[s], (uint32_t)ring.phase))) {
+        dead = true;
+        abort_now();
+      }
+      const uint8_t* cs = codes_s + s * UB * BOX_BYTES;
+      const uint8_t* hs = hib_s + s * L::HIB_BYTES;
+      const uint32_t xs_base = smem_u32(x_s + s * L::X_BYTES);
+      for (int bi = 0; bi < BPU; ++bi, bw = (bw + 1 == NWG) ? 0 : bw + 1) {
+        if (bw != wg) continue;
+        const int ds = dr.slot;
+        if (!dead) {
+          // the accumulator slot was read and re-zeroed by the epilogue, and the
+          // previous batch's MMAs (which read the A slot) are complete
+          bool ok = mbar_wait(&d_empty[wg * 2 + ds], (uint32_t)(dr.phase ^ 1));
+          if (ok && prev_slot >= 0) ok = mbar_wait(&d_full[wg * 2 + prev_slot], (uint32_t)prev_phase);
+          if (!__all_sync(0xffffffffu, ok)) {
+            dead = true;
+            abort_now();
+          }
+        }
+        if (!dead) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int g = 0; g < GB; ++g) {
+            const int gi = bi * GB + g;  // group within the unit
+            uint32_t v[C::ACOLS];
+            dequant_group<FMT>(cs + (gi / Tr::GPB) * BOX_BYTES, hs + r * 32 * UB + (gi / Tr::GPB) * 32 - r * 32,
+                               r, gi % Tr::GPB, v);
+            if constexpr (C::ACOLS == 32)
+              tmem_st_x32(a_base + lane_ofs + g * C::ACOLS, v);
+            else
+              tmem_st_x16(a_base + lane_ofs + g * C::ACOLS, v);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        named_barrier_sync(1 + wg, 128);
+        if (issuer && !dead) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int g = 0; g < GB; ++g) {
+            const int kofs = (bi * GB + g) * Tr::GK;  // K offset of the group inside the unit
+            const uint32_t xaddr = xs_base + (kofs / 64) * TP * 128 + (kofs % 64) * 2;
+#pragma unroll
+            for (int kk = 0; kk < Tr::GK / 16; ++kk)
+              mma_f16_ts(d_base + ds * C::D_COLS + g * TP, a_base + g * C::ACOLS + kk * 8,
+                         sdesc_k_sw128(xaddr + kk * 32), idesc, 1u);
+          }
+          tc_commit(&d_full[wg * 2 + ds]);
+        }
+        prev_slot = ds;
+        prev_phase = dr.phase;
+        dr.next(2);
+      }
+      ring.next(NS);
     }
-  } else if (warp >= W_EPI0 && warp < W_EPI0 + 4) {
+  } else if (warp >= W_EPI0) {
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int et = threadIdx.x - W_EPI0 * 32;  // 0..127
@@ -382,63 +444,75 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     float acc[TP];
 #pragma unroll
     for (int t = 0; t < TP; ++t) acc[t] = 0.0f;
-    int64_t D = 0;
     bool dead = false;  // after a timed-out wait: skip waits and work, keep the barrier sequence
-    for (int64_t u = u0; u < u1; ++u) {
-      const int64_t cu = u - u0;
-      const int s = (int)(cu % NS);
-      const int64_t tile = u / args.cpt, ch = u % args.cpt;
-      const int64_t row = tile * 128 + r;
-      const int gcount = (int)min((int64_t)Tr::GPC, ng - ch * Tr::GPC);
-      const bool seg_first = (u == u0) || ch == 0;
-      const bool seg_last = (u + 1 == u1) || ((u + 1) % args.cpt == 0);
+    Ring ring{0, 0};
+    Ring dr[NWG] = {{0, 0}, {0, 0}};
+    int bw = 0;
+    int tile = tile0, ch = ch0;
+    for (int cu = 0; cu < nunits; ++cu) {
+      const int s = ring.slot;
+      const int64_t row = (int64_t)tile * 128 + r;
+      const bool seg_first = cu == 0 || ch == 0;
+      const bool seg_last = cu + 1 == nunits || ch == cpt - 1;
       if (seg_first) {
 #pragma unroll
         for (int t = 0; t < TP; ++t) acc[t] = 0.0f;
       }
       dead = dead || __any_sync(0xffffffffu, *abort_flag != 0);
       // the stage's scales have landed once its barrier completed (acquire)
-      if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)((cu / NS) & 1)))) {
+      if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)ring.phase))) {
         dead = true;
         abort_now();
       }
-      const __half* sc_row = (const __half*)(sc_s + s * C::SC_BYTES) + r * Tr::GPC;
-      for (int gi = 0; gi < gcount; ++gi) {
-        const bool close_acc = Tr::PER_GROUP || (seg_last && gi == gcount - 1);
-        if (!close_acc) continue;
-        const int d = (int)(D % ND);
-        const uint32_t dpar = (uint32_t)((D / ND) & 1);
-        ++D;
+      const __half* sc_row = (const __half*)(sc_s + s * L::SC_BYTES) + r * GPC;
+      for (int bi = 0; bi < BPU; ++bi, bw = (bw + 1 == NWG) ? 0 : bw + 1) {
+        const int ds = dr[bw].slot;
+        const uint32_t dph = (uint32_t)dr[bw].phase;
+        dr[bw].next(2);
         if (dead) continue;
-        float sc = 1.0f;
-        if constexpr (Tr::PER_GROUP) sc = __half2float(sc_row[gi]);
-        if (!__all_sync(0xffffffffu, mbar_wait(&d_full[d], dpar))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&d_full[bw * 2 + ds], dph))) {
           dead = true;
           abort_now();
           continue;
         }
         tc_fence_after();
+        const uint32_t d_addr = tmem + bw * C::WG_COLS + C::A_COLS + ds * C::D_COLS + lane_ofs;
 #pragma unroll
-        for (int c = 0; c < TP; c += 16) {
-          if (c < T) {
-            uint32_t vr[16];
-            tmem_ld_x16(tmem_d + lane_ofs + d * TP + c, vr);
-            tmem_ld_wait();
+        for (int g = 0; g < GB; ++g) {
+          float sc = 1.0f;
+          if constexpr (Tr::PER_GROUP) sc = __half2float(sc_row[bi * GB + g]);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc[c + j] = fmaf(sc, __uint_as_float(vr[j]), acc[c + j]);
+          for (int c = 0; c < TP; c += 16) {
+            if (c < T) {
+              uint32_t vr[16];
+              tmem_ld_x16(d_addr + g * TP + c, vr);
+              tmem_ld_wait();
+              tmem_fill_x16(d_addr + g * TP + c, 0u);  // ready for a later batch
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[c + j] = fmaf(sc, __uint_as_float(vr[j]), acc[c + j]);
+            }
           }
         }
+        tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&d_empty[d]);
+        mbar_arrive(&d_empty[bw * 2 + ds]);
       }
-      if (!dead) mbar_arrive(&empty[s]);
+      // every batch of the unit is done: the TMA stage (codes, activations,
+      // scales) can be refilled
+      if (!dead && et == 0) mbar_arrive(&empty[s]);
+      ring.next(NS);
+      const int cur_tile = tile;
+      if (++ch == cpt) {
+        ch = 0;
+        ++tile;
+      }
       if (!seg_last) continue;
       // ---- the CTA's part of this tile is complete
       float rs = 1.0f;
       if constexpr (FMT == QLIN_FP8_ROW) {
         if (row < args.n) rs = __bfloat162float(((const __nv_bfloat16*)args.scales)[row]);
       }
-      const int64_t tstart = tile * args.cpt, tend = tstart + args.cpt;
+      const int64_t tstart = (int64_t)cur_tile * cpt, tend = tstart + cpt;
       const bool whole = u0 <= tstart && u1 >= tend;
       if (whole) {
         if (!dead && row < args.n) {
@@ -455,7 +529,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         continue;
       }
       // split tile: publish this part, the last contributor reduces
-      const int slot = (tile == u0 / args.cpt) ? 0 : 1;
+      const int slot = (cur_tile == tile0) ? 0 : 1;
       float* mine = args.partials + ((int64_t)blockIdx.x * 2 + slot) * T * 128;
       if (!dead) {
 #pragma unroll
@@ -463,9 +537,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (t < T) mine[t * 128 + et] = acc[t];
       }
       __threadfence();
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      if (et == 0) *fix_slot = dead ? -1 : atomicAdd(&args.counters[tile], 1);
-      asm volatile("bar.sync 2, 128;" ::: "memory");
+      named_barrier_sync(15, 128);
+      if (et == 0) *fix_slot = dead ? -1 : atomicAdd(&args.counters[cur_tile], 1);
+      named_barrier_sync(15, 128);
       const int old = *fix_slot;
       const int64_t i_first = unit_owner(tstart, U, P), i_last = unit_owner(tend - 1, U, P);
       if (old == (int)(i_last - i_first)) {
@@ -473,7 +547,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
         for (int t = 0; t < TP; ++t) acc[t] = 0.0f;
         for (int64_t i = i_first; i <= i_last; ++i) {
-          const int si = (tile == unit_start(i, U, P) / args.cpt) ? 0 : 1;
+          const int si = (cur_tile == unit_start(i, U, P) / cpt) ? 0 : 1;
           const float* part = args.partials + (i * 2 + si) * T * 128;
 #pragma unroll
           for (int t = 0; t < TP; ++t)
@@ -490,45 +564,48 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
         }
-        if (et == 0) args.counters[tile] = 0;  // leave the counter ready for the next call
+        if (et == 0) args.counters[cur_tile] = 0;  // leave the counter ready for the next call
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == W_MMA) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
-template <int FMT>
-int64_t chunk_k() {
-  return TcT<FMT>::KC;
-}
+int tpad_of(int64_t t) { return t <= 16 ? 16 : t <= 32 ? 32 : t <= 48 ? 48 : 64; }
 
-int64_t tc_chunk_k(int fmt) {
-  switch (fmt) {
-    case QLIN_Q4_G64: return TcT<QLIN_Q4_G64>::KC;
-    case QLIN_Q5_G64: return TcT<QLIN_Q5_G64>::KC;
-    case QLIN_Q8_G32: return TcT<QLIN_Q8_G32>::KC;
-    case QLIN_FP8_ROW: return TcT<QLIN_FP8_ROW>::KC;
-    default: return TcT<QLIN_BF16>::KC;
+template <int FMT>
+int unit_k_fmt(int tp) {
+  switch (tp) {
+    case 16: return Cfg<FMT, 16>::KC;
+    case 32: return Cfg<FMT, 32>::KC;
+    case 48: return Cfg<FMT, 48>::KC;
+    default: return Cfg<FMT, 64>::KC;
   }
 }
 
-int tpad_of(int64_t t) { return t <= 16 ? 16 : t <= 32 ? 32 : t <= 48 ? 48 : 64; }
+int unit_k(int fmt, int tp) {
+  switch (fmt) {
+    case QLIN_Q4_G64: return unit_k_fmt<QLIN_Q4_G64>(tp);
+    case QLIN_Q5_G64: return unit_k_fmt<QLIN_Q5_G64>(tp);
+    case QLIN_Q8_G32: return unit_k_fmt<QLIN_Q8_G32>(tp);
+    case QLIN_FP8_ROW: return unit_k_fmt<QLIN_FP8_ROW>(tp);
+    default: return unit_k_fmt<QLIN_BF16>(tp);
+  }
+}
 
 template <int FMT, int TP>
 int launch_tp(const CUtensorMap& mc, const CUtensorMap& mh, const CUtensorMap& mx, const TcArgs& a,
               int grid, cudaStream_t st) {
   using C = Cfg<FMT, TP>;
-  static_assert(C::NS >= 2, "pipeline needs two stages");
-  static_assert(NA * C::ACOLS + ND * TP <= (int)TMEM_COLS, "tensor memory budget");
   auto kern = gemv_tc_kernel<FMT, TP>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-  kern<<<grid, TC_THREADS, C::SMEM, st>>>(mc, mh, mx, a);
+  kern<<<grid, THREADS, C::SMEM, st>>>(mc, mh, mx, a);
   return cuda_status(cudaGetLastError());
 }
 
@@ -545,13 +622,11 @@ int launch_fmt(int tp, const CUtensorMap& mc, const CUtensorMap& mh, const CUten
 
 }  // namespace
 
-// Q4/Q5 need whole 256-column chunks (8-byte scale rows per chunk), Q8 whole
-// 128-column chunks; other shapes take the CUDA-core kernel.
+// Rows must be whole units (K a multiple of the unit's K columns: 512 for
+// Q4/Q5 at T <= 16, etc.); other shapes take the CUDA-core kernel.
 bool gemv_tc_supported(const qlin_weights& w, int64_t t) {
   if (t < 1 || t > 64) return false;
-  if ((w.fmt == QLIN_Q4_G64 || w.fmt == QLIN_Q5_G64) && w.k % 256 != 0) return false;
-  if (w.fmt == QLIN_Q8_G32 && w.k % 128 != 0) return false;
-  return true;
+  return w.k % unit_k(w.fmt, tpad_of(t)) == 0;
 }
 
 size_t gemv_tc_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
@@ -562,12 +637,12 @@ size_t gemv_tc_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
 
 int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                    const Exec& ex) {
+  const int tp = tpad_of(t);
   const int64_t tiles = (w.n + 127) / 128;
-  const int64_t kc = tc_chunk_k(w.fmt);
-  const int64_t cpt = (w.k + kc - 1) / kc;
+  const int64_t kc = unit_k(w.fmt, tp);
+  const int64_t cpt = w.k / kc;
   const int64_t units = tiles * cpt;
   const int grid = (int)std::min<int64_t>(ex.num_sms, units);
-  const int tp = tpad_of(t);
   const int64_t row_bytes = w.fmt == QLIN_Q4_G64 || w.fmt == QLIN_Q5_G64 ? w.k / 2
                             : w.fmt == QLIN_BF16                      ? w.k * 2
                                                                       : w.k;
@@ -579,8 +654,10 @@ int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
                       (uint64_t)w.k * 2, 64, (uint32_t)tp, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   if (w.fmt == QLIN_Q5_G64) {
+    // high-bit plane: 32 bytes per row per 128-byte box of codes
+    const uint32_t hib_box = (uint32_t)(32 * (kc / 256));
     rc = encode_tmap_2d(&mh, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.hibits, (uint64_t)(w.k / 8),
-                        (uint64_t)w.n, (uint64_t)(w.k / 8), 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+                        (uint64_t)w.n, (uint64_t)(w.k / 8), hib_box, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
   } else {
     mh = mc;

@@ -190,6 +190,21 @@ def test_gemv_small_shapes(fmt, t):
     check_gemv(pw, ref, x, q.OUT_F32)
 
 
+@pytest.mark.parametrize("fmt", list(FMTS))
+@pytest.mark.parametrize("t", [1, 3, 16, 17, 33, 48, 64])
+def test_gemv_tensor_core_path_split_tiles(fmt, t):
+    """K = 1536 is whole units for every format, so the tensor-core kernel runs;
+    200 rows x 3 units per tile over 6 CTAs splits every tile three ways."""
+    n, k = 200, 1536
+    w = synth.weights_f32(n, k, seed=600 + t)
+    x = synth.activations_bf16(t, k, seed=700 + t)
+    ref = oracle.pack(FMTS[fmt], w.numpy())
+    pw = pack_gpu(FMTS[fmt], w.to(DEV))
+    check_gemv(pw, ref, x, q.OUT_F32)
+    # a second call on the same workspace: the split-tile counters were left at zero
+    check_gemv(pw, ref, x, q.OUT_BF16)
+
+
 @pytest.mark.parametrize("fmt", ["q4", "q5", "fp8"])
 def test_gemv_bf16_output_and_long_k(fmt):
     n, k, t = 96, 17408, 2
