@@ -7,22 +7,26 @@
 // B200 design:
 //   * quantize_act_kernel: one warp per (token, 128 columns); lanes 0-15 and
 //     16-31 each own one 64-group; amax by shuffles, IEEE division, RNE.
-//   * gemm_a8_kernel: one CTA per 128 weight rows x 128 tokens.
-//       - a TMA warp streams the packed weight codes (raw nibbles), the int8
-//         activation codes and (for Q5) the high-bit plane into a 2-stage ring
-//         of 256-column chunks (four 64-groups);
-//       - four unpack warps expand the nibbles to signed int8 directly into the
-//         128-byte-swizzled K-major operand layout the tensor core reads;
-//       - one thread issues tcgen05.mma.kind::i8 (M=128, N=128, K=32) twice per
-//         group into a fresh int32 accumulator in tensor memory, double-buffered
-//         so the tensor core runs one group ahead of the epilogue;
-//       - eight epilogue warps (two column halves x four lane quarters) read
-//         each group's int32 sums with tcgen05.ld and apply
-//         y += FP32(ws * as) * float(S) in registers; the output tile is
-//         written once at the end.
-//   The tensor core is idle part of the time: every group sum needs FP32 work
-//   on the CUDA cores (the method's per-group promotion), which bounds this
-//   kernel below the int8 tensor peak.
+//   * gemm_a8_kernel: persistent, one CTA per SM walking 128-row x 128-token
+//     tiles (neighbouring CTAs share weight rows; the activations stay in L2):
+//       - a TMA warp streams the packed weight codes, the int8 activation codes
+//         and (Q5) the high-bit plane into a 4-stage ring of 256-column chunks
+//         (four 64-groups), its lanes cp.async the stage's scales;
+//       - four unpack warps (one per tensor-memory lane quarter, thread = row)
+//         expand each group's nibbles to signed int8 and write them with
+//         tcgen05.st into an 8-slot ring of A operands in tensor memory;
+//       - one thread issues tcgen05.mma.kind::i8 (A in tensor memory, B = the
+//         activation codes in shared memory, M = 128, N = 128, K = 32) twice
+//         per group into one of two group-sum slots, pre-armed with a bias so
+//         that one FP32 subtraction turns the sum into a float;
+//       - eight epilogue warps read each group's sums with tcgen05.ld and do
+//         y += FP32(ws * as) * S, y itself being an FP32 tile in tensor memory
+//         (keeps registers free), then write y once per tile.
+//   Every group sum needs three FP32 operations on the CUDA cores (the
+//   method's per-group promotion), which bounds this kernel below the int8
+//   tensor peak.
+#include <algorithm>
+
 #include "qlin_internal.cuh"
 
 namespace qlin {
@@ -69,19 +73,28 @@ __global__ void quantize_act_kernel(const uint16_t* __restrict__ x, int64_t t, i
 // ---------------------------------------------------------------------------
 // Int8 group-sum GEMM.
 // ---------------------------------------------------------------------------
-constexpr int BM = 128;         // weight rows per CTA (tensor-memory lanes)
-constexpr int BN = 128;         // tokens per CTA (accumulator columns)
+constexpr int BM = 128;         // weight rows per tile (tensor-memory lanes)
+constexpr int BN = 128;         // tokens per tile (accumulator columns)
 constexpr int BKC = 256;        // K columns per pipeline stage (four 64-groups)
 constexpr int GPS = BKC / 64;   // groups per stage
-constexpr int STAGES = 2;
+constexpr int STAGES = 4;
+constexpr int NDS = 2;          // group-sum slots (128 columns each)
+constexpr int NAS = 8;          // A slots (one group of int8 codes: 16 columns each)
+constexpr int Y_COL0 = NDS * BN;        // the tile's FP32 output accumulator (128 columns)
+constexpr int A_COL0 = Y_COL0 + BN;
 constexpr int NUM_EPI_WARPS = 8;
-constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_UNPACK0 = 10;
-constexpr int NUM_UNPACK_THREADS = 64;  // two warps, two weight rows per thread
-constexpr int NUM_THREADS = 12 * 32;
+// warp w accesses tensor-memory lanes 32 * (w % 4) ..: four consecutive warps
+// cover all 128 rows
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_UNPACK0 = 4, WARP_EPI0 = 8;
+constexpr int NUM_THREADS = 16 * 32;
+// Accumulators start at this bit pattern (FP32 1.5 * 2^23): after the integer
+// MMAs add a group sum S (|S| < 2^22) the word reads as the float 1.5 * 2^23 + S,
+// so one FP32 subtraction recovers S exactly.
+constexpr uint32_t ACC_BIAS = 0x4B400000u;
+constexpr float ACC_BIAS_F = 12582912.0f;
 
 struct __align__(1024) StageSmem {
-  uint8_t a[2][BM * 128];        // int8 weights, two 128-column swizzled atoms
-  uint8_t b[2][BN * 128];        // int8 activations, two atoms
+  uint8_t b[2][BN * 128];        // int8 activations, two 128-column swizzled atoms
   uint8_t raw[BM * 128];         // packed nibbles of 256 columns (swizzled)
   uint8_t hib[BM * 32];          // Q5 high bits of 256 columns
   float xsb[GPS * BN];           // activation scales of the stage, [group][token]
@@ -90,8 +103,9 @@ struct __align__(1024) StageSmem {
 
 struct Smem {
   StageSmem st[STAGES];
-  uint64_t full[STAGES], a_ready[STAGES], empty[STAGES];
-  uint64_t d_full[2], d_empty[2], drain;
+  uint64_t full[STAGES], empty[STAGES];
+  uint64_t a_full[NAS], a_free[NAS];
+  uint64_t d_full[NDS], d_empty[NDS];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -103,8 +117,9 @@ struct GemmArgs {
   int32_t* sums_dbg;
   int32_t* dev_status;
   int64_t n, k, t;
+  int64_t tiles_t;       // token tiles
+  int64_t tiles;         // row tiles x token tiles
   int y_dtype;
-  int debug;
 };
 
 __device__ __forceinline__ void set_abort(Smem& sm, int32_t* dev_status) {
@@ -112,6 +127,17 @@ __device__ __forceinline__ void set_abort(Smem& sm, int32_t* dev_status) {
   report_timeout(dev_status);
 }
 __device__ __forceinline__ bool aborted(Smem& sm) { return *(volatile int*)&sm.abort_flag != 0; }
+
+// A ring position: slot index and the parity of its current use.
+struct Ring {
+  int slot, phase;
+  __device__ __forceinline__ void next(int n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1;
+    }
+  }
+};
 
 // Expand 8 nibbles of one layout word into 8 signed int8 codes in element order.
 template <int BITS>
@@ -144,27 +170,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((void*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t0 = (int64_t)blockIdx.x * BN;
-  const int64_t n0 = (int64_t)blockIdx.y * BM;
   const int64_t ng = args.k / 64;
-  const int64_t nchunks = (args.k + BKC - 1) / BKC;
+  const int nchunks = (int)((args.k + BKC - 1) / BKC);
+  // tiles of this CTA: blockIdx.x, + gridDim.x, ...; tile i covers rows
+  // (i / tiles_t) * BM and tokens (i % tiles_t) * BN (neighbouring CTAs share
+  // weight rows, the activations stay in L2)
+  const int64_t my_tiles = (args.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.full[s], 1 + 32);  // TMA issue + 32 scale-copy arrivals
-      mbar_init(&sm.a_ready[s], NUM_UNPACK_THREADS);
-      mbar_init(&sm.empty[s], 1 + NUM_EPI_WARPS * 32);
+      mbar_init(&sm.full[s], 1 + 32);                 // TMA issue + 32 scale-copy arrivals
+      mbar_init(&sm.empty[s], 4 + 1 + NUM_EPI_WARPS);  // unpack warps, MMA commit, epilogue warps
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.d_full[b], 1);
-      mbar_init(&sm.d_empty[b], NUM_EPI_WARPS * 32);
+    for (int j = 0; j < NAS; ++j) {
+      mbar_init(&sm.a_full[j], 4);  // unpack warps
+      mbar_init(&sm.a_free[j], 1);  // MMA commit
     }
-    mbar_init(&sm.drain, 1);
+    for (int d = 0; d < NDS; ++d) {
+      mbar_init(&sm.d_full[d], 1);
+      mbar_init(&sm.d_empty[d], NUM_EPI_WARPS);
+    }
     sm.abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == WARP_MMA) {
-    tmem_alloc(&sm.tmem_base, 256);
+    tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
   if (warp == WARP_TMA && lane == 0) {
@@ -176,212 +206,279 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  if (warp >= WARP_EPI0) {  // arm every group-sum slot with the bias; zero the output accumulator
+    const int quarter = warp & 3, half = (warp - WARP_EPI0) >> 2;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    for (int d = 0; d < NDS; ++d)
+      for (int c = 0; c < 64; c += 32) tmem_fill_x32(tmem + lo + d * BN + half * 64 + c, ACC_BIAS);
+    for (int c = 0; c < 64; c += 32) tmem_fill_x32(tmem + lo + Y_COL0 + half * 64 + c, 0u);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp == WARP_TMA) {
     // lane 0 issues the TMA copies; all 32 lanes copy the stage's weight and
     // activation scales into shared memory with cp.async (same barrier).
     // The activations come from the quantizer kernel launched just before.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    int64_t issued = 0;
-    for (int64_t kc = 0; kc < nchunks; ++kc) {
-      const int s = (int)(kc % STAGES);
-      const uint32_t par = (uint32_t)((kc / STAGES) & 1);
-      if (!__all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.empty[s], par ^ 1))) {
-        if (lane == 0) set_abort(sm, args.dev_status);
-        break;
-      }
-      const int gcount = (int)min((int64_t)GPS, ng - kc * GPS);
-      if (lane == 0) {
-        uint32_t bytes = BM * 128 + 2 * BN * 128 + (BITS == 5 ? BM * 32 : 0);
-        mbar_arrive_expect_tx(&sm.full[s], bytes);
-        tma_load_2d(sm.st[s].raw, &tm_codes, &sm.full[s], (int)(kc * 128), (int)n0);
-        if (BITS == 5) tma_load_2d(sm.st[s].hib, &tm_hib, &sm.full[s], (int)(kc * 32), (int)n0);
-        tma_load_2d(sm.st[s].b[0], &tm_act, &sm.full[s], (int)(kc * BKC), (int)t0);
-        tma_load_2d(sm.st[s].b[1], &tm_act, &sm.full[s], (int)(kc * BKC + 128), (int)t0);
-      }
-      // weight scales: two groups (4 bytes) per copy; K % 128 == 0 keeps them aligned
-      for (int rr = lane; rr < BM; rr += 32) {
-        const int64_t grow = n0 + rr;
-        if (grow < args.n)
-          for (int gp = 0; gp < gcount; gp += 2)
-            cp_async_4(&sm.st[s].wsb[rr * GPS + gp], args.ws + grow * ng + kc * GPS + gp);
-      }
-      // activation scales, [group][token]
-      for (int tt = lane; tt < BN; tt += 32) {
-        const int64_t gt = t0 + tt;
-        if (gt < args.t)
-          for (int gi = 0; gi < gcount; ++gi)
-            cp_async_4(&sm.st[s].xsb[gi * BN + tt], args.xs + gt * ng + kc * GPS + gi);
-      }
-      cp_async_arrive_noinc(&sm.full[s]);
-      ++issued;
-    }
-    // let every copy in flight land before the CTA can leave
-    if (lane == 0)
-      for (int64_t kc = issued > STAGES ? issued - STAGES : 0; kc < issued; ++kc)
-        mbar_wait(&sm.full[kc % STAGES], (uint32_t)((kc / STAGES) & 1));
-  } else if (warp == WARP_MMA) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_i8(BM, BN);
-      int64_t G = 0;
-      for (int64_t kc = 0; kc < nchunks && !aborted(sm); ++kc) {
-        const int s = (int)(kc % STAGES);
-        const uint32_t par = (uint32_t)((kc / STAGES) & 1);
-        if (!mbar_wait(&sm.full[s], par) || !mbar_wait(&sm.a_ready[s], par)) {
-          set_abort(sm, args.dev_status);
-          break;
-        }
-        tc_fence_after();
-        const int gcount = (int)min((int64_t)GPS, ng - kc * GPS);
-        bool ok = true;
-        for (int gi = 0; gi < gcount; ++gi, ++G) {
-          const int b = (int)(G & 1);
-          if (!mbar_wait(&sm.d_empty[b], (uint32_t)(((G >> 1) & 1) ^ 1))) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(sm.st[s].a[gi >> 1]) + (gi & 1) * 64;
-          const uint32_t b_base = smem_u32(sm.st[s].b[gi >> 1]) + (gi & 1) * 64;
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_i8_ss(tmem + b * BN, sdesc_k_sw128(a_base + kk * 32), sdesc_k_sw128(b_base + kk * 32),
-                      idesc, kk);
-          tc_commit(&sm.d_full[b]);
-        }
-        if (!ok) { set_abort(sm, args.dev_status); break; }
-        tc_commit(&sm.empty[s]);
-      }
-      tc_commit(&sm.drain);
-      mbar_wait(&sm.drain, 0);
-    }
-  } else if (warp >= WARP_UNPACK0) {
-    const int ut = threadIdx.x - WARP_UNPACK0 * 32;  // rows ut and ut + 64 of the tile
-    for (int64_t kc = 0; kc < nchunks; ++kc) {
-      const int s = (int)(kc % STAGES);
-      const uint32_t par = (uint32_t)((kc / STAGES) & 1);
-      if (aborted(sm)) break;
-      if (!mbar_wait(&sm.full[s], par)) { set_abort(sm, args.dev_status); break; }
-      const uint8_t* raw = sm.st[s].raw;
-#pragma unroll 1
-      for (int rr = 0; rr < 2; ++rr) {
-        const int r = ut + 64 * rr;
-        uint32_t hw[8];
-        if (BITS == 5) {
-          const uint4* hp = (const uint4*)(sm.st[s].hib + r * 32);
-          uint4 h0 = hp[0], h1 = hp[1];
-          hw[0] = h0.x; hw[1] = h0.y; hw[2] = h0.z; hw[3] = h0.w;
-          hw[4] = h1.x; hw[5] = h1.y; hw[6] = h1.z; hw[7] = h1.w;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {  // 16-byte unit u of the row = 32 elements
-          uint4 c = *(const uint4*)(raw + sw128_offset(r, u));
-          uint32_t wv[4] = {c.x, c.y, c.z, c.w};
-          uint32_t o[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t h = 0;
-            if (BITS == 5) h = hw[u] >> (4 * j);
-            uint2 e = expand_word<BITS>(wv[j], h);
-            o[2 * j] = e.x;
-            o[2 * j + 1] = e.y;
-          }
-          uint8_t* arow = sm.st[s].a[u >> 2];
-          const uint32_t unit0 = (u & 3) * 2;
-          *(uint4*)(arow + sw128_offset(r, unit0)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *(uint4*)(arow + sw128_offset(r, unit0 + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
-        }
-      }
-      fence_async_smem();
-      mbar_arrive(&sm.a_ready[s]);
-    }
-  } else {
-    // ---- epilogue: warps 0..7; warp w reads lanes 32*(w%4).., columns 64*(w/4)..
-    const int quarter = warp & 3, half = warp >> 2;
-    const int row = quarter * 32 + lane;
-    const int64_t grow = n0 + row;
-    const int col0 = half * 64;
-    float acc[64];
-#pragma unroll
-    for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
-    int64_t G = 0;
-    for (int64_t kc = 0; kc < nchunks; ++kc) {
-      const int s = (int)(kc % STAGES);
-      const int gcount = (int)min((int64_t)GPS, ng - kc * GPS);
-      // acquire the stage (its scale copies landed when the barrier completed)
-      if (__any_sync(0xffffffffu, aborted(sm)) ||
-          !__all_sync(0xffffffffu, mbar_wait(&sm.full[s], (uint32_t)((kc / STAGES) & 1)))) {
-        set_abort(sm, args.dev_status);
-        break;
-      }
-      const float* xsb = sm.st[s].xsb;
-      const uint2 wsr = *(const uint2*)(&sm.st[s].wsb[row * GPS]);
-      const float ws0 = __low2float(*(const __half2*)&wsr.x), ws1 = __high2float(*(const __half2*)&wsr.x);
-      const float ws2 = __low2float(*(const __half2*)&wsr.y), ws3 = __high2float(*(const __half2*)&wsr.y);
-      bool ok = true;
-      for (int gi = 0; gi < gcount; ++gi, ++G) {
-        const int b = (int)(G & 1);
-        const float wsc = gi == 0 ? ws0 : gi == 1 ? ws1 : gi == 2 ? ws2 : ws3;
-        // warp-uniform: tcgen05.ld below needs the whole warp
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.d_full[b], (uint32_t)((G >> 1) & 1)))) {
+    int issued = 0;
+    Ring ring{0, 0};
+    bool ok = true;
+    for (int64_t it = 0; it < my_tiles && ok; ++it) {
+      const int64_t tile = blockIdx.x + it * gridDim.x;
+      const int64_t n0 = (tile / args.tiles_t) * BM, t0 = (tile % args.tiles_t) * BN;
+      for (int kc = 0; kc < nchunks; ++kc) {
+        const int s = ring.slot;
+        if (!__all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.empty[s], (uint32_t)(ring.phase ^ 1)))) {
+          if (lane == 0) set_abort(sm, args.dev_status);
           ok = false;
           break;
         }
-        tc_fence_after();
-        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + b * BN + col0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sv[32];
-          tmem_ld_x32(taddr + 32 * h, sv);
-          tmem_ld_wait();
-          if (h == 1) {
-            tc_fence_before();
-            mbar_arrive(&sm.d_empty[b]);
-          }
-          if (DEBUG && grow < args.n) {
-            int32_t* dp = args.sums_dbg + ((t0 + col0 + 32 * h) * args.n + grow) * ng + kc * GPS + gi;
-            const int64_t dstep = args.n * ng;
-#pragma unroll
-            for (int j = 0; j < 32; ++j, dp += dstep)
-              if (t0 + col0 + 32 * h + j < args.t) *dp = (int32_t)sv[j];
-          }
-          const float4* xv4 = (const float4*)(xsb + gi * BN + col0 + 32 * h);
-#pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 xv = xv4[j4];
-            const int j = 4 * j4;
-            acc[32 * h + j] = fmaf(wsc * xv.x, (float)(int32_t)sv[j], acc[32 * h + j]);
-            acc[32 * h + j + 1] = fmaf(wsc * xv.y, (float)(int32_t)sv[j + 1], acc[32 * h + j + 1]);
-            acc[32 * h + j + 2] = fmaf(wsc * xv.z, (float)(int32_t)sv[j + 2], acc[32 * h + j + 2]);
-            acc[32 * h + j + 3] = fmaf(wsc * xv.w, (float)(int32_t)sv[j + 3], acc[32 * h + j + 3]);
-          }
+        const int gcount = (int)min((int64_t)GPS, ng - (int64_t)kc * GPS);
+        if (lane == 0) {
+          uint32_t bytes = BM * 128 + 2 * BN * 128 + (BITS == 5 ? BM * 32 : 0);
+          mbar_arrive_expect_tx(&sm.full[s], bytes);
+          tma_load_2d(sm.st[s].raw, &tm_codes, &sm.full[s], kc * 128, (int)n0);
+          if (BITS == 5) tma_load_2d(sm.st[s].hib, &tm_hib, &sm.full[s], kc * 32, (int)n0);
+          tma_load_2d(sm.st[s].b[0], &tm_act, &sm.full[s], kc * BKC, (int)t0);
+          tma_load_2d(sm.st[s].b[1], &tm_act, &sm.full[s], kc * BKC + 128, (int)t0);
         }
+        // weight scales: two groups (4 bytes) per copy; K % 128 == 0 keeps them aligned
+        for (int rr = lane; rr < BM; rr += 32) {
+          const int64_t grow = n0 + rr;
+          if (grow < args.n)
+            for (int gp = 0; gp < gcount; gp += 2)
+              cp_async_4(&sm.st[s].wsb[rr * GPS + gp], args.ws + grow * ng + (int64_t)kc * GPS + gp);
+        }
+        // activation scales, [group][token]
+        for (int tt = lane; tt < BN; tt += 32) {
+          const int64_t gt = t0 + tt;
+          if (gt < args.t)
+            for (int gi = 0; gi < gcount; ++gi)
+              cp_async_4(&sm.st[s].xsb[gi * BN + tt], args.xs + gt * ng + (int64_t)kc * GPS + gi);
+        }
+        cp_async_arrive_noinc(&sm.full[s]);
+        ++issued;
+        ring.next(STAGES);
+      }
+    }
+    // let every copy in flight land before the CTA can leave
+    if (lane == 0) {
+      Ring r2{0, 0};
+      for (int i = 0; i < issued; ++i) {
+        if (i + STAGES >= issued) mbar_wait(&sm.full[r2.slot], (uint32_t)r2.phase);
+        r2.next(STAGES);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_i8(BM, BN);
+      Ring ring{0, 0}, ar{0, 0}, dr{0, 0};
+      bool ok = true;
+      for (int64_t it = 0; it < my_tiles && ok; ++it) {
+        for (int kc = 0; kc < nchunks && ok; ++kc) {
+          const int s = ring.slot;
+          ok = !aborted(sm) && mbar_wait(&sm.full[s], (uint32_t)ring.phase);
+          const int gcount = (int)min((int64_t)GPS, ng - (int64_t)kc * GPS);
+          for (int gi = 0; gi < gcount && ok; ++gi) {
+            ok = mbar_wait(&sm.a_full[ar.slot], (uint32_t)ar.phase) &&
+                 mbar_wait(&sm.d_empty[dr.slot], (uint32_t)(dr.phase ^ 1)) && !aborted(sm);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t b_base = smem_u32(sm.st[s].b[gi >> 1]) + (gi & 1) * 64;
+            const uint32_t a_col = tmem + A_COL0 + ar.slot * 16;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_i8_ts(tmem + dr.slot * BN, a_col + kk * 8, sdesc_k_sw128(b_base + kk * 32), idesc, 1u);
+            tc_commit(&sm.a_free[ar.slot]);
+            tc_commit(&sm.d_full[dr.slot]);
+            ar.next(NAS);
+            dr.next(NDS);
+          }
+          if (ok) tc_commit(&sm.empty[s]);  // the activation tile is free once these MMAs finish
+          ring.next(STAGES);
+        }
+      }
+      if (!ok) set_abort(sm, args.dev_status);
+    }
+    __syncwarp();
+  } else if (warp >= WARP_UNPACK0 && warp < WARP_EPI0) {
+    // ---- unpack: thread = weight row; nibbles (+ high bits) -> signed int8
+    // codes written with tcgen05.st as the MMA's A operand, one group per A slot
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_ofs = (uint32_t)(quarter * 32) << 16;
+    Ring ring{0, 0}, ar{0, 0};
+    bool ok = true;
+    for (int64_t it = 0; it < my_tiles && ok; ++it) {
+      for (int kc = 0; kc < nchunks; ++kc) {
+        const int s = ring.slot;
+        if (!__all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.full[s], (uint32_t)ring.phase))) {
+          if (lane == 0) set_abort(sm, args.dev_status);
+          ok = false;
+          break;
+        }
+        const int gcount = (int)min((int64_t)GPS, ng - (int64_t)kc * GPS);
+        const uint8_t* raw = sm.st[s].raw;
+        for (int gi = 0; gi < gcount; ++gi) {
+          // the MMAs that last read this A slot are complete
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.a_free[ar.slot], (uint32_t)(ar.phase ^ 1)))) {
+            if (lane == 0) set_abort(sm, args.dev_status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint2 hw = make_uint2(0, 0);  // Q5: the high-bit words of units 2gi, 2gi+1
+          if (BITS == 5) hw = *(const uint2*)(sm.st[s].hib + r * 32 + gi * 8);
+          uint32_t o[16];
+#pragma unroll
+          for (int uu = 0; uu < 2; ++uu) {  // 16-byte units 2gi, 2gi+1 of the row = 64 elements
+            const int u = 2 * gi + uu;
+            const uint4 c = *(const uint4*)(raw + sw128_offset(r, u));
+            const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t h = 0;
+              if (BITS == 5) h = (uu ? hw.y : hw.x) >> (4 * j);
+              const uint2 e = expand_word<BITS>(wv[j], h);
+              o[8 * uu + 2 * j] = e.x;
+              o[8 * uu + 2 * j + 1] = e.y;
+            }
+          }
+          tmem_st_x16(tmem + lane_ofs + A_COL0 + ar.slot * 16, o);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.a_full[ar.slot]);
+          ar.next(NAS);
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[s]);  // codes and high bits consumed
+        ring.next(STAGES);
+      }
+    }
+  } else if (warp >= WARP_EPI0) {
+    // ---- epilogue: warp w reads lanes 32*(w%4).., token columns 64*half..; the
+    // tile's FP32 accumulator y lives in tensor memory next to the group sums:
+    // per group and 16-column chunk, y += FP32(ws * as) * S
+    const int quarter = warp & 3, half = (warp - WARP_EPI0) >> 2;
+    const int row = quarter * 32 + lane;
+    const int col0 = half * 64;
+    const uint32_t lane_ofs = (uint32_t)(quarter * 32) << 16;
+    const uint32_t yaddr = tmem + lane_ofs + Y_COL0 + col0;
+    Ring ring{0, 0}, dr{0, 0};
+    bool ok = true;
+    for (int64_t it = 0; it < my_tiles && ok; ++it) {
+      const int64_t tile = blockIdx.x + it * gridDim.x;
+      const int64_t n0 = (tile / args.tiles_t) * BM, t0 = (tile % args.tiles_t) * BN;
+      const int64_t grow = n0 + row;
+      for (int kc = 0; kc < nchunks && ok; ++kc) {
+        const int s = ring.slot;
+        const int gcount = (int)min((int64_t)GPS, ng - (int64_t)kc * GPS);
+        // acquire the stage (its scale copies landed when the barrier completed)
+        if (__any_sync(0xffffffffu, aborted(sm)) ||
+            !__all_sync(0xffffffffu, mbar_wait(&sm.full[s], (uint32_t)ring.phase))) {
+          ok = false;
+          break;
+        }
+        const float* xsb = sm.st[s].xsb;
+        const uint2 wsr = *(const uint2*)(&sm.st[s].wsb[row * GPS]);
+        for (int gi = 0; gi < gcount; ++gi) {
+          const uint32_t wsw = (gi & 2) ? wsr.y : wsr.x;
+          const float wsc = __half2float(__ushort_as_half((unsigned short)(wsw >> ((gi & 1) * 16))));
+          // warp-uniform: tcgen05.ld below needs the whole warp
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.d_full[dr.slot], (uint32_t)dr.phase))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t saddr = tmem + lane_ofs + dr.slot * BN + col0;
+#pragma unroll 1
+          for (int h = 0; h < 4; ++h) {
+            uint32_t sv[16], yv[16];
+            tmem_ld_x16(saddr + 16 * h, sv);
+            tmem_ld_x16(yaddr + 16 * h, yv);
+            tmem_ld_wait();
+            tmem_fill_x16(saddr + 16 * h, ACC_BIAS);  // re-arm for a later group
+            if (DEBUG && grow < args.n) {
+              int32_t* dp = args.sums_dbg + ((t0 + col0 + 16 * h) * args.n + grow) * ng + (int64_t)kc * GPS + gi;
+              const int64_t dstep = args.n * ng;
+#pragma unroll
+              for (int j = 0; j < 16; ++j, dp += dstep)
+                if (t0 + col0 + 16 * h + j < args.t) *dp = (int32_t)(sv[j] - ACC_BIAS);
+            }
+            const float4* xv4 = (const float4*)(xsb + gi * BN + col0 + 16 * h);
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const float4 xv = xv4[j4];
+              const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = 4 * j4 + e;
+                yv[j] = __float_as_uint(
+                    fmaf(wsc * xa[e], __uint_as_float(sv[j]) - ACC_BIAS_F, __uint_as_float(yv[j])));
+              }
+            }
+            tmem_st_x16(yaddr + 16 * h, yv);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.d_empty[dr.slot]);
+          dr.next(NDS);
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[s]);  // the stage's scales are consumed
+        ring.next(STAGES);
       }
       if (!ok) {
         set_abort(sm, args.dev_status);
         break;
       }
-      mbar_arrive(&sm.empty[s]);
-    }
-    if (!__any_sync(0xffffffffu, aborted(sm)) && grow < args.n) {
-      const int64_t base = (t0 + col0) * args.n + grow;
+      // the tile is complete: write y, zero the accumulator for the next tile
       const int jmax = (int)min((int64_t)64, args.t - (t0 + col0));
-      if (args.y_dtype == QLIN_OUT_F32) {
-        float* yp = (float*)args.y + base;
+#pragma unroll 1
+      for (int h = 0; h < 4; ++h) {
+        uint32_t yv[16];
+        tmem_ld_x16(yaddr + 16 * h, yv);
+        tmem_ld_wait();
+        tmem_fill_x16(yaddr + 16 * h, 0u);
+        if (grow < args.n) {
+          const int64_t base = (t0 + col0 + 16 * h) * args.n + grow;
+          if (args.y_dtype == QLIN_OUT_F32) {
+            float* yp = (float*)args.y + base;
 #pragma unroll
-        for (int j = 0; j < 64; ++j, yp += args.n)
-          if (j < jmax) *yp = acc[j];
-      } else {
-        __nv_bfloat16* yp = (__nv_bfloat16*)args.y + base;
+            for (int j = 0; j < 16; ++j, yp += args.n)
+              if (16 * h + j < jmax) *yp = __uint_as_float(yv[j]);
+          } else {
+            __nv_bfloat16* yp = (__nv_bfloat16*)args.y + base;
 #pragma unroll
-        for (int j = 0; j < 64; ++j, yp += args.n)
-          if (j < jmax) *yp = __float2bfloat16_rn(acc[j]);
+            for (int j = 0; j < 16; ++j, yp += args.n)
+              if (16 * h + j < jmax) *yp = __float2bfloat16_rn(__uint_as_float(yv[j]));
+          }
+        }
       }
+      tmem_st_wait();
     }
   }
 
+  // Every group's completion was observed by the epilogue before this point,
+  // so no MMA is in flight -- unless a wait timed out; then give the tensor
+  // core ample time (1 ms) before the tensor memory is released.
   tc_fence_before();
   __syncthreads();
   if (warp == WARP_MMA) {
+    if (aborted(sm)) {
+      const unsigned long long t0 = global_ns();
+      while (global_ns() - t0 < 1000000ull) {
+      }
+    }
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -442,12 +539,14 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
   args.n = n;
   args.k = k;
   args.t = t;
+  args.tiles_t = (t + BN - 1) / BN;
+  args.tiles = args.tiles_t * ((n + BM - 1) / BM);
   args.y_dtype = y_dtype;
-  args.debug = (flags & QLIN_DEBUG_GROUP_SUMS) ? 1 : 0;
+  const bool debug = (flags & QLIN_DEBUG_GROUP_SUMS) != 0;
 
   const size_t smem = sizeof(Smem) + 1024;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((t + BN - 1) / BN), (unsigned)((n + BM - 1) / BM));
+  cfg.gridDim = dim3((unsigned)std::min<int64_t>(args.tiles, ex.num_sms));
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = ex.stream;
@@ -457,8 +556,8 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  auto kern = w.fmt == QLIN_Q4_G64 ? (args.debug ? gemm_a8_kernel<4, true> : gemm_a8_kernel<4, false>)
-                                    : (args.debug ? gemm_a8_kernel<5, true> : gemm_a8_kernel<5, false>);
+  auto kern = w.fmt == QLIN_Q4_G64 ? (debug ? gemm_a8_kernel<4, true> : gemm_a8_kernel<4, false>)
+                                    : (debug ? gemm_a8_kernel<5, true> : gemm_a8_kernel<5, false>);
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   e = cudaLaunchKernelEx(&cfg, kern, tm_codes, tm_hib, tm_act, args);
   return cuda_status(e);

@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&empty[s], 1);      // released by the epilogue once the unit is done
     }
     for (int i = 0; i < 2 * NWG; ++i) {
-      mbar_init(&d_full[i], 1);
+      mbar_init(&d_full[i], C::GB);  // one tcgen05.commit per issuing warp
       mbar_init(&d_empty[i], 128);
     }
     *abort_flag = 0;
@@ -360,7 +360,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_ofs = (uint32_t)(quarter * 32) << 16;
-    const bool issuer = quarter == 0 && lane == 0;
     const uint32_t idesc = idesc_bf16(128, TP);
     const uint32_t a_base = tmem + wg * C::WG_COLS;
     const uint32_t d_base = a_base + C::A_COLS;
@@ -417,17 +416,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_before();
         named_barrier_sync(1 + wg, 128);
-        if (issuer && !dead) {
+        // warp q issues group q of the batch from lane 0: one thread issues an
+        // MMA only every ~45-80 cycles, threads of different warps in parallel
+        if (quarter < GB && lane == 0 && !dead) {
           tc_fence_after();
-#pragma unroll 1
-          for (int g = 0; g < GB; ++g) {
-            const int kofs = (bi * GB + g) * Tr::GK;  // K offset of the group inside the unit
-            const uint32_t xaddr = xs_base + (kofs / 64) * TP * 128 + (kofs % 64) * 2;
+          const int g = quarter;
+          const int kofs = (bi * GB + g) * Tr::GK;  // K offset of the group inside the unit
+          const uint32_t xaddr = xs_base + (kofs / 64) * TP * 128 + (kofs % 64) * 2;
 #pragma unroll
-            for (int kk = 0; kk < Tr::GK / 16; ++kk)
-              mma_f16_ts(d_base + ds * C::D_COLS + g * TP, a_base + g * C::ACOLS + kk * 8,
-                         sdesc_k_sw128(xaddr + kk * 32), idesc, 1u);
-          }
+          for (int kk = 0; kk < Tr::GK / 16; ++kk)
+            mma_f16_ts(d_base + ds * C::D_COLS + g * TP, a_base + g * C::ACOLS + kk * 8,
+                       sdesc_k_sw128(xaddr + kk * 32), idesc, 1u);
           tc_commit(&d_full[wg * 2 + ds]);
         }
         prev_slot = ds;

@@ -160,11 +160,13 @@ def test_quantize_act_bit_exact(shape):
 # ---------------------------------------------------------------------------
 # BF16-route GEMV
 # ---------------------------------------------------------------------------
-def check_gemv(pw, ref, x, y_dtype=q.OUT_F32):
+def check_gemv(pw, ref, x, y_dtype=q.OUT_F32, ws=None):
     t = x.shape[0]
     y = torch.empty(t, pw.n, dtype=torch.float32 if y_dtype == q.OUT_F32 else torch.bfloat16,
                     device=DEV)
-    ws = q.Workspace(DEV).ensure(q.qlin_gemv_workspace_bytes(pw, t))
+    if ws is None:
+        ws = q.Workspace(DEV)
+    ws.ensure(q.qlin_gemv_workspace_bytes(pw, t))
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     q.qlin_gemv(pw, x.to(DEV), y, y_dtype, workspace=ws, dev_status=status)
     yr, br = oracle.gemv(ref, bits16(x), nthreads=8)
@@ -200,9 +202,12 @@ def test_gemv_tensor_core_path_split_tiles(fmt, t):
     x = synth.activations_bf16(t, k, seed=700 + t)
     ref = oracle.pack(FMTS[fmt], w.numpy())
     pw = pack_gpu(FMTS[fmt], w.to(DEV))
-    check_gemv(pw, ref, x, q.OUT_F32)
+    ws = q.Workspace(DEV)
+    check_gemv(pw, ref, x, q.OUT_F32, ws=ws)
     # a second call on the same workspace: the split-tile counters were left at zero
-    check_gemv(pw, ref, x, q.OUT_BF16)
+    check_gemv(pw, ref, x, q.OUT_BF16, ws=ws)
+    counters = ws.buffer[: ((n + 127) // 128) * 4]
+    assert not counters.any()
 
 
 @pytest.mark.parametrize("fmt", ["q4", "q5", "fp8"])
@@ -239,7 +244,10 @@ def test_gemv_full_size_sampled_rows(name, fmt, n, k, t):
     pw = pack_gpu(fmt, w)
     y = torch.empty(t, n, dtype=torch.float32, device=DEV)
     ws = q.Workspace(DEV).ensure(q.qlin_gemv_workspace_bytes(pw, t))
-    q.qlin_gemv(pw, x, y, q.OUT_F32, workspace=ws)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q.qlin_gemv(pw, x, y, q.OUT_F32, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0  # no on-chip wait ran out
     g = torch.Generator().manual_seed(1)
     rows = torch.cat([torch.randperm(n, generator=g)[:61], torch.tensor([0, n - 1])])
     ref = oracle.pack(fmt, w[rows.to(DEV)].cpu().numpy())
@@ -254,6 +262,32 @@ def test_gemv_full_size_sampled_rows(name, fmt, n, k, t):
         if ref[key] is not None:
             assert np.array_equal(sub[key][rows.numpy()], ref[key]), key
     del got_packed
+
+
+@pytest.mark.parametrize("fmt", list(FMTS))
+@pytest.mark.parametrize("t", [1, 17, 33, 64])
+def test_gemv_several_units_per_cta(fmt, t):
+    """4096 x 4096: every CTA walks several units, so each ring and barrier of
+    the pipeline goes through several phases; sampled rows against the oracle
+    and no on-chip wait may run out."""
+    n, k = 4096, 4096
+    w = synth.weights_f32(n, k, seed=800 + t, device=DEV)
+    x = synth.activations_bf16(t, k, seed=900 + t)
+    pw = pack_gpu(FMTS[fmt], w)
+    y = torch.empty(t, n, dtype=torch.float32, device=DEV)
+    ws = q.Workspace(DEV).ensure(q.qlin_gemv_workspace_bytes(pw, t))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for _ in range(2):
+        q.qlin_gemv(pw, x.to(DEV), y, q.OUT_F32, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    g = torch.Generator().manual_seed(t)
+    rows = torch.cat([torch.randperm(n, generator=g)[:45], torch.tensor([0, 127, 128, n - 1])])
+    ref = oracle.pack(FMTS[fmt], w[rows.to(DEV)].cpu().numpy())
+    yr, br = oracle.gemv(ref, bits16(x), nthreads=8)
+    got = y[:, rows.to(DEV)].cpu().numpy().astype(np.float64)
+    bad = np.abs(got - yr) > 1e-3 * br
+    assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
 
 
 # ---------------------------------------------------------------------------
