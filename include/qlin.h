@@ -200,6 +200,25 @@ QLIN_API int qlin_gemm_a8(const qlin_weights* w, const uint16_t* x_bf16, const i
                  int64_t t, void* y, int y_dtype, uint32_t flags, int32_t* group_sums_dbg,
                  const qlin_exec* ex);
 
+/* qlin_gemv without a caller workspace.  The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory when they
+ * call (memory planned once at start-up; plain C code owning only w, x and y).
+ * Same arguments, results, limits and errors as qlin_gemv (stream is a
+ * cudaStream_t or NULL, dev_status as qlin_exec.dev_status, may be NULL); the
+ * scratch qlin_gemv would take from qlin_exec.workspace comes instead from a
+ * fixed 16 MiB device array inside the library, one per device.
+ * Requests whose qlin_gemv_workspace_bytes() exceeds 16 MiB return
+ * QLIN_ERR_WORKSPACE (T <= 64 on the quantized formats always fits; BF16
+ * weights at large T * N may not).
+ * The first call on a device resolves the array's address and zero-fills it
+ * (synchronously); make that first call before any stream capture.  Each call
+ * clears the array's split-tile counters on `stream` before its kernels.
+ * The array is shared by all calls on a device: calls that may overlap in time
+ * (other streams or host threads) race on it and must be serialized by the
+ * caller.  Allocates nothing. */
+QLIN_API int qlin_gemv_noalloc(const qlin_weights* w, const uint16_t* x_bf16, int64_t t, void* y,
+                               int y_dtype, void* stream, int32_t* dev_status);
+
 #ifdef __cplusplus
 }
 #endif

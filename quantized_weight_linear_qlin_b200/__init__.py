@@ -17,7 +17,7 @@ __all__ = [
     "ALLOW_A8", "DEBUG_GROUP_SUMS", "PackedWeights", "Workspace", "lib",
     "qlin_packed_bytes", "qlin_pack_weights", "qlin_decode_mxfp8", "qlin_quantize_act",
     "qlin_gemv", "qlin_gemv_workspace_bytes", "qlin_gemm_a8", "qlin_gemm_a8_workspace_bytes",
-    "qlin_status_string",
+    "qlin_status_string", "qlin_gemv_noalloc",
 ]
 
 Q4_G64, Q5_G64, Q8_G32, FP8_ROW, BF16 = 0, 1, 2, 3, 4
@@ -33,7 +33,7 @@ LIB_PATH = os.path.join(HERE, "libqlin.so")
 EXPORTED = (
     "qlin_status_string", "qlin_packed_bytes", "qlin_pack_weights", "qlin_decode_mxfp8",
     "qlin_quantize_act", "qlin_gemv_workspace_bytes", "qlin_gemv",
-    "qlin_gemm_a8_workspace_bytes", "qlin_gemm_a8",
+    "qlin_gemm_a8_workspace_bytes", "qlin_gemm_a8", "qlin_gemv_noalloc",
 )
 
 
@@ -73,6 +73,7 @@ def lib():
         L.qlin_quantize_act.argtypes = [vp, i64, i64, vp, vp, C.POINTER(_Exec)]
         L.qlin_gemv_workspace_bytes.argtypes = [C.POINTER(_Weights), i64, vp]
         L.qlin_gemv.argtypes = [C.POINTER(_Weights), vp, i64, vp, i32, C.POINTER(_Exec)]
+        L.qlin_gemv_noalloc.argtypes = [C.POINTER(_Weights), vp, i64, vp, i32, vp, vp]
         L.qlin_gemm_a8_workspace_bytes.argtypes = [i64, i64, i64, vp]
         L.qlin_gemm_a8.argtypes = [C.POINTER(_Weights), vp, vp, vp, i64, vp, i32, u32, vp,
                                    C.POINTER(_Exec)]
@@ -200,6 +201,17 @@ def qlin_gemv(w: PackedWeights, x, y, y_dtype=OUT_BF16, workspace=None, stream=N
     d = w.desc()
     e = _exec(stream, workspace, dev_status)
     _check(lib().qlin_gemv(C.byref(d), _ptr(x), t, _ptr(y), y_dtype, C.byref(e)), "qlin_gemv")
+    return y
+
+
+def qlin_gemv_noalloc(w: PackedWeights, x, y, y_dtype=OUT_BF16, stream=None, dev_status=None):
+    """qlin_gemv with the library's fixed device scratch instead of a workspace."""
+    t = x.shape[0]
+    d = w.desc()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    _check(lib().qlin_gemv_noalloc(C.byref(d), _ptr(x), t, _ptr(y), y_dtype, C.c_void_p(stream.cuda_stream),
+                                   None if dev_status is None else _ptr(dev_status)), "qlin_gemv_noalloc")
     return y
 
 
