@@ -396,12 +396,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t saddr = tmem + lane_ofs + dr.slot * BN + col0;
-#pragma unroll 1
+          // four 16-column chunks, software-pipelined: chunk h+1's tensor-memory
+          // loads are in flight while chunk h is computed
+          uint32_t s0[16], y0[16], s1[16], y1[16];
+          tmem_ld_x16(saddr, s0);
+          tmem_ld_x16(yaddr, y0);
+#pragma unroll
           for (int h = 0; h < 4; ++h) {
-            uint32_t sv[16], yv[16];
-            tmem_ld_x16(saddr + 16 * h, sv);
-            tmem_ld_x16(yaddr + 16 * h, yv);
+            uint32_t* sv = (h & 1) ? s1 : s0;
+            uint32_t* yv = (h & 1) ? y1 : y0;
             tmem_ld_wait();
+            if (h < 3) {
+              tmem_ld_x16(saddr + 16 * (h + 1), (h & 1) ? s0 : s1);
+              tmem_ld_x16(yaddr + 16 * (h + 1), (h & 1) ? y0 : y1);
+            }
             tmem_fill_x16(saddr + 16 * h, ACC_BIAS);  // re-arm for a later group
             if (DEBUG && grow < args.n) {
               int32_t* dp = args.sums_dbg + ((t0 + col0 + 16 * h) * args.n + grow) * ng + (int64_t)kc * GPS + gi;
