@@ -105,13 +105,31 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
 // T <= 64 runs on the tensor cores; BF16 weights at prefill sizes (T > 64)
 // and Q5 rows whose high-bit plane is not 16-byte aligned per row use the
 // CUDA-core kernel.
+// BF16 weights at more than 64 tokens (the GDN a/b projection at prefill):
+// the tensor-core kernel in 64-token chunks, one after the other on the stream
+// (the weights, 1 MB for 96 x 5120, stay in L2 between chunks).
+constexpr int64_t kTcMaxT = 64;
+static bool bf16_chunked(const qlin_weights& w, int64_t t) {
+  return w.fmt == QLIN_BF16 && t > kTcMaxT && gemv_tc_supported(w, kTcMaxT);
+}
+
 size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
+  if (bf16_chunked(w, t)) return gemv_tc_workspace_bytes(w, kTcMaxT, num_sms);
   if (gemv_tc_supported(w, t)) return gemv_tc_workspace_bytes(w, t, num_sms);
   return gemv_cc_workspace_bytes(w, t);
 }
 
 int launch_gemv(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                 const Exec& ex) {
+  if (bf16_chunked(w, t)) {
+    const size_t ysz = y_dtype == QLIN_OUT_F32 ? 4 : 2;
+    for (int64_t t0 = 0; t0 < t; t0 += kTcMaxT) {
+      const int64_t tc = t - t0 < kTcMaxT ? t - t0 : kTcMaxT;
+      const int rc = launch_gemv_tc(w, x + t0 * w.k, tc, (uint8_t*)y + (size_t)t0 * w.n * ysz, y_dtype, ex);
+      if (rc != QLIN_OK) return rc;
+    }
+    return QLIN_OK;
+  }
   if (gemv_tc_supported(w, t)) return launch_gemv_tc(w, x, t, y, y_dtype, ex);
   return launch_gemv_cc(w, x, t, y, y_dtype, ex, (float*)ex.workspace);
 }

@@ -220,9 +220,11 @@ def test_gemv_bf16_output_and_long_k(fmt):
     check_gemv(pw, ref, x, q.OUT_BF16)
 
 
-def test_gemv_bf16_weights_prefill_sizes():
-    # GDN a/b projection kept in BF16: 96 x 5120 at a prefill chunk
-    n, k, t = 96, 5120, 512
+@pytest.mark.parametrize("t", [130, 512])
+def test_gemv_bf16_weights_prefill_sizes(t):
+    # GDN a/b projection kept in BF16: 96 x 5120 at a prefill chunk (64-token
+    # tensor-core launches; 130 leaves a ragged last chunk)
+    n, k = 96, 5120
     w = synth.weights_f32(n, k, seed=9)
     x = synth.activations_bf16(t, k, seed=10)
     ref = oracle.pack(q.BF16, w.numpy())
