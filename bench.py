@@ -358,14 +358,24 @@ def run_ours(args, dist):
     e2e_ms = dist.max(s2.elapsed_time(e2))
     e2e_value = dist.sum(step_bytes * args.steps) / (e2e_ms / 1e3) / 1e9
 
-    # dominant kernel of the step (largest share of the device time in the
-    # launch list): the tensor-core GEMV instantiation that serves gate+up at
-    # T = 1 and 4 (Q4, T padded to 16); calls 0 and 2 of every step
-    dom_ms = sum(timer.pairs[8 * i + j][0].elapsed_time(timer.pairs[8 * i + j][1])
-                 for i in range(args.steps) for j in (0, 2)) / args.steps
-    dom_bytes = gemv_bytes(copies[0][0], 1) + gemv_bytes(copies[0][0], 4)
-    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-    traffic = measured_traffic("gemv_tc_q4_gate_up_34816x5120_T4")
+    # dominant kernel of the step: the kernel instantiation with the largest
+    # summed device time over the step's 8 calls (call j of a step: matrix
+    # j % 2 = gate+up / down, T = T_LIST[j // 2])
+    groups = {}
+    for j in range(2 * len(T_LIST)):
+        t = T_LIST[j // 2]
+        fmt = "Q4_G64" if j % 2 == 0 else "Q5_G64"
+        kern = (f"gemv_sm_kernel<{fmt}, 1>" if t == 1 else
+                f"gemv_tc_kernel<{fmt}, {16 if t <= 16 else 32 if t <= 32 else 48 if t <= 48 else 64}>")
+        ms_j = sum(timer.pairs[8 * i + j][0].elapsed_time(timer.pairs[8 * i + j][1])
+                   for i in range(args.steps)) / args.steps
+        g = groups.setdefault(kern, {"ms": 0.0, "bytes": 0, "calls": []})
+        g["ms"] += ms_j
+        g["bytes"] += gemv_bytes(copies[0][j % 2], t)
+        g["calls"].append(("gate+up 34816x5120" if j % 2 == 0 else "down 5120x17408") + f" T={t}")
+    dom_kern, dom = max(groups.items(), key=lambda kv: kv[1]["ms"])
+    achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+    traffic = measured_traffic(dom_kern)
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -388,9 +398,10 @@ def run_ours(args, dist):
             "timed_region": "CUDA graph replay of the step's 8 launches",
         },
         "roofline": {
-            "bound": "hbm", "kernel": "gemv_tc_kernel<Q4_G64, T padded to 16>: gate+up 34816x5120 at T=1 and T=4",
+            "bound": "hbm", "kernel": dom_kern + ": " + ", ".join(dom["calls"]),
             "timing": "CUDA events around each call, calls queued behind a device spin",
-            "algorithmic_bytes_per_launch": dom_bytes / 2,
+            "algorithmic_bytes_per_launch": dom["bytes"] / len(dom["calls"]),
+            "share_of_step": round(dom["ms"] / call_ms, 3),
             "achieved": round(achieved, 1), "peak": hbm, "peak_kind": f"{peak_kind} HBM copy GB/s",
             "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic,
             "step_achieved_all_8_calls": round(step_bytes / (call_ms / 1e3) / 1e9, 1),

@@ -12,6 +12,10 @@ size_t gemv_cc_workspace_bytes(const qlin_weights& w, int64_t t);
 int launch_gemv_cc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                    const Exec& ex, float* acc_ws);
 bool gemv_tc_supported(const qlin_weights& w, int64_t t);
+bool gemv_sm_supported(const qlin_weights& w, int64_t t);
+size_t gemv_sm_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
+int launch_gemv_sm(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
+                   const Exec& ex);
 size_t gemv_tc_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
 int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                    const Exec& ex);
@@ -114,6 +118,7 @@ static bool bf16_chunked(const qlin_weights& w, int64_t t) {
 }
 
 size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
+  if (gemv_sm_supported(w, t)) return gemv_sm_workspace_bytes(w, t, num_sms);
   if (bf16_chunked(w, t)) return gemv_tc_workspace_bytes(w, kTcMaxT, num_sms);
   if (gemv_tc_supported(w, t)) return gemv_tc_workspace_bytes(w, t, num_sms);
   return gemv_cc_workspace_bytes(w, t);
@@ -121,6 +126,8 @@ size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
 
 int launch_gemv(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                 const Exec& ex) {
+  // T = 1: CUDA-core kernel (mixed-precision FMA); T <= 64: tensor cores
+  if (gemv_sm_supported(w, t)) return launch_gemv_sm(w, x, t, y, y_dtype, ex);
   if (bf16_chunked(w, t)) {
     const size_t ysz = y_dtype == QLIN_OUT_F32 ? 4 : 2;
     for (int64_t t0 = 0; t0 < t; t0 += kTcMaxT) {

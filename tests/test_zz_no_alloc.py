@@ -47,10 +47,11 @@ def test_noalloc_matches_workspace_path_twice(fmt, n, k, t):
 
 
 def test_noalloc_rejects_requests_beyond_the_array():
-    # BF16 weights at T > 64 run on the CUDA-core kernel; with K beyond its
-    # 2048-column stage it splits K and needs a T * N FP32 accumulator:
-    # 32 MiB here, above the 16 MiB array
-    n, k, t = 4096, 4096, 2048
+    # BF16 weights whose K is not a whole number of tensor-core units run on
+    # the general CUDA-core kernel; with K beyond its 2048-column stage it
+    # splits K and needs a T * N FP32 accumulator: 32 MiB here, above the
+    # 16 MiB array
+    n, k, t = 4096, 4160, 2048
     pw = q.PackedWeights(q.BF16, n, k, device=DEV)
     x = torch.zeros(t, k, dtype=torch.bfloat16, device=DEV)
     y = torch.empty(t, n, dtype=torch.bfloat16, device=DEV)
