@@ -102,11 +102,17 @@ def _ptr(t):
     return C.c_void_p(t.data_ptr())
 
 
+def _current_stream_handle():
+    """cudaStream_t of torch's current stream on the current device."""
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return raw(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
+
+
 def _exec(stream=None, workspace=None, dev_status=None):
-    if stream is None:
-        stream = torch.cuda.current_stream()
     e = _Exec()
-    e.stream = C.c_void_p(stream.cuda_stream)
+    e.stream = C.c_void_p(_current_stream_handle() if stream is None else stream.cuda_stream)
     e.dev_status = None if dev_status is None else _ptr(dev_status)
     if workspace is not None:
         buf = workspace.buffer if isinstance(workspace, Workspace) else workspace
@@ -141,12 +147,17 @@ class PackedWeights:
             torch.empty(sb, dtype=torch.uint8, device=device) if sb else None)
 
     def desc(self):
-        d = _Weights()
-        d.fmt, d.flags, d.n, d.k = self.fmt, self.flags, self.n, self.k
-        d.codes = _ptr(self.codes)
-        d.hibits = None if self.hibits is None else _ptr(self.hibits)
-        d.scales = None if self.scales is None else _ptr(self.scales)
-        return d
+        """The qlin_weights descriptor (built once; rebuilt if a buffer is replaced)."""
+        key = (self.codes.data_ptr(), None if self.hibits is None else self.hibits.data_ptr(),
+               None if self.scales is None else self.scales.data_ptr(), self.flags)
+        if getattr(self, "_desc_key", None) != key:
+            d = _Weights()
+            d.fmt, d.flags, d.n, d.k = self.fmt, self.flags, self.n, self.k
+            d.codes = _ptr(self.codes)
+            d.hibits = None if self.hibits is None else _ptr(self.hibits)
+            d.scales = None if self.scales is None else _ptr(self.scales)
+            self._desc, self._desc_key = d, key
+        return self._desc
 
     def bytes(self):
         return sum(t.numel() * t.element_size() for t in (self.codes, self.hibits, self.scales)
@@ -208,9 +219,8 @@ def qlin_gemv_noalloc(w: PackedWeights, x, y, y_dtype=OUT_BF16, stream=None, dev
     """qlin_gemv with the library's fixed device scratch instead of a workspace."""
     t = x.shape[0]
     d = w.desc()
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    _check(lib().qlin_gemv_noalloc(C.byref(d), _ptr(x), t, _ptr(y), y_dtype, C.c_void_p(stream.cuda_stream),
+    sh = _current_stream_handle() if stream is None else stream.cuda_stream
+    _check(lib().qlin_gemv_noalloc(C.byref(d), _ptr(x), t, _ptr(y), y_dtype, C.c_void_p(sh),
                                    None if dev_status is None else _ptr(dev_status)), "qlin_gemv_noalloc")
     return y
 

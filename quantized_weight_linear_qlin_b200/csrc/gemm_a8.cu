@@ -5,8 +5,8 @@
 // activation_scale in FP32.
 //
 // B200 design:
-//   * quantize_act_kernel: one warp per (token, 128 columns); lanes 0-15 and
-//     16-31 each own one 64-group; amax by shuffles, IEEE division, RNE.
+//   * quantize_act_kernel: eight lanes per (token, 64-group), 16-byte loads;
+//     amax by shuffles, IEEE division, RNE.
 //   * gemm_a8_kernel: persistent, one CTA per SM walking 128-row x 128-token
 //     tiles (neighbouring CTAs share weight rows; the activations stay in L2):
 //       - a TMA warp streams the packed weight codes, the int8 activation codes
@@ -35,37 +35,47 @@ namespace {
 // ---------------------------------------------------------------------------
 // Activation quantizer.
 // ---------------------------------------------------------------------------
-__global__ void quantize_act_kernel(const uint16_t* __restrict__ x, int64_t t, int64_t k,
+// Eight lanes per 64-group (8 elements = 16 bytes each), four groups per warp;
+// x is [T][K] with K % 64 == 0, so group g covers elements [64g, 64g + 64) of
+// the flattened array and its scale is xs[g].
+__global__ void quantize_act_kernel(const uint16_t* __restrict__ x, int64_t groups,
                                     int8_t* __restrict__ xq, float* __restrict__ xs) {
   // let the GEMM that consumes these codes start its prologue now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
-  const int64_t chunks = (k + 127) / 128;
-  const int64_t items = t * chunks;
-  const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x / 32);
-  for (int64_t it = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); it < items;
-       it += warps_total) {
-    const int64_t tt = it / chunks, ch = it % chunks;
-    const int64_t e0 = ch * 128 + 4 * lane;
-    const bool valid = e0 < k;  // k % 64 == 0: a 16-lane half is valid or not as a whole
-    uint2 raw = make_uint2(0, 0);
-    if (valid) raw = __ldcs((const uint2*)(x + tt * k + e0));
-    float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
-                  __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
-    float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-#pragma unroll
-    for (int o = 8; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const float s = __fdiv_rn(a, 127.0f);
-    uint32_t packed = 0;
+  const int64_t total = groups * 8;  // 8 lanes per group
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // whole warps iterate together (the shuffles need every lane)
+  for (int64_t wbase = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); wbase < total; wbase += stride) {
+    const int64_t idx = wbase + lane;
+    const bool valid = idx < total;  // total % 8 == 0: a group is valid or not as a whole
+    const int64_t e0 = idx * 8;
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (valid) raw = __ldcs((const uint4*)(x + e0));
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    float v[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+    // the 8 lanes of a group are consecutive and aligned to 8 within the warp
+#pragma unroll
+    for (int o = 4; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const float sc = __fdiv_rn(a, 127.0f);
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
       int q = 0;
-      if (s != 0.0f) q = (int)fminf(fmaxf(rintf(__fdiv_rn(v[i], s)), -127.0f), 127.0f);
-      packed |= ((uint32_t)q & 0xFFu) << (8 * i);
+      if (sc != 0.0f) q = (int)fminf(fmaxf(rintf(__fdiv_rn(v[i], sc)), -127.0f), 127.0f);
+      packed[i >> 2] |= ((uint32_t)q & 0xFFu) << (8 * (i & 3));
     }
     if (valid) {
-      __stcg((uint32_t*)(xq + tt * k + e0), packed);
-      if ((lane & 15) == 0) xs[tt * (k / 64) + e0 / 64] = s;
+      __stcg((uint2*)(xq + e0), make_uint2(packed[0], packed[1]));
+      if ((lane & 7) == 0) xs[idx >> 3] = sc;
     }
   }
 }
@@ -502,12 +512,13 @@ size_t gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, int num_sms) {
 
 int launch_quantize_act(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* xs,
                         const Exec& ex) {
-  const int64_t items = t * ((k + 127) / 128);
-  int64_t blocks = (items + 7) / 8;
-  const int64_t cap = (int64_t)ex.num_sms * 16;
+  const int64_t groups = t * (k / 64);
+  const int64_t threads = groups * 8;
+  int64_t blocks = (threads + 511) / 512;
+  const int64_t cap = (int64_t)ex.num_sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  quantize_act_kernel<<<(unsigned)blocks, 256, 0, ex.stream>>>(x, t, k, xq, xs);
+  quantize_act_kernel<<<(unsigned)blocks, 512, 0, ex.stream>>>(x, groups, xq, xs);
   return cuda_status(cudaGetLastError());
 }
 

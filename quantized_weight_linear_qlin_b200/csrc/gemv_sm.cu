@@ -325,7 +325,8 @@ int launch_t(const CUtensorMap& mc, const CUtensorMap& mh, const CUtensorMap& mx
              int grid, cudaStream_t st) {
   using C = SmCfg<FMT, T>;
   auto kern = gemv_sm_kernel<FMT, T>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  const cudaError_t e = set_smem_once<gemv_sm_kernel<FMT, T>>((int)C::SMEM);
+  if (e != cudaSuccess) return cuda_status(e);
   kern<<<grid, SM_THREADS, C::SMEM, st>>>(mc, mh, mx, a);
   return cuda_status(cudaGetLastError());
 }

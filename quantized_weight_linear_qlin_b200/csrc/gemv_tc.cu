@@ -465,7 +465,8 @@ int launch_tp(const CUtensorMap& mc, const CUtensorMap& mh, const CUtensorMap& m
               int grid, cudaStream_t st) {
   using C = Cfg<FMT, TP>;
   auto kern = gemv_tc_kernel<FMT, TP>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  const cudaError_t e = set_smem_once<gemv_tc_kernel<FMT, TP>>((int)C::SMEM);
+  if (e != cudaSuccess) return cuda_status(e);
   kern<<<grid, THREADS, C::SMEM, st>>>(mc, mh, mx, a);
   return cuda_status(cudaGetLastError());
 }

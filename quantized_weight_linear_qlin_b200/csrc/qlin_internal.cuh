@@ -9,6 +9,7 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "qlin.h"
@@ -48,6 +49,20 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
                    uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA; }
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device
+// (a host-side call that would otherwise run on every launch).
+template <auto Kern>
+inline cudaError_t set_smem_once(int bytes) {
+  static std::atomic<unsigned long long> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // ---------------------------------------------------------------------------
 // Device helpers.
