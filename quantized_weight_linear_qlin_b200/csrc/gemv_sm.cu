@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
         const uint8_t* st = base + s * C::STAGE;
         const uint8_t* xs = st + C::OFF_X;
         const __half* sc_row = (const __half*)(st + C::OFF_SC) + r * GPC;
-#pragma unroll 1
+#pragma unroll 2
         for (int gg = 0; gg < GPC / 2; ++gg) {
           const int gi = h * (GPC / 2) + gg;  // group within the unit
           uint32_t v[C::ACOLS];

@@ -188,47 +188,69 @@ __device__ __forceinline__ uint32_t bf16x2_mul_rn(uint32_t a, uint32_t b) {
   return d;
 }
 
-__global__ void decode_mxfp8_kernel(const uint4* __restrict__ words, const uint8_t* __restrict__ sc,
-                                    int64_t chunks, uint4* __restrict__ out) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const uint4 w = __ldcs(words + i);
-    const uint32_t b = sc[i >> 1];  // cols % 32 == 0: chunk i lies in scale block i / 2
-    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-    // a byte with (c & 0x7F) == 0x7F is a NaN code
-    uint32_t nan_bytes = 0;
+__device__ __forceinline__ void decode_chunk(const uint4 w, uint32_t b, uint4* __restrict__ out) {
+  const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+  // a byte with (c & 0x7F) == 0x7F is a NaN code
+  uint32_t nan_bytes = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t y = (wv[j] & 0x7F7F7F7Fu) ^ 0x7F7F7F7Fu;  // zero byte where the code is NaN
+    nan_bytes |= (y - 0x01010101u) & ~y & 0x80808080u;
+  }
+  uint32_t o[8];
+  if (nan_bytes == 0 && b != 255) {
+    const uint32_t e = b == 0 ? 0x0040u : (b << 7);  // BF16 2^(b-127) (2^-127 is subnormal)
+    const uint32_t scale2 = e | (e << 16);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t y = (wv[j] & 0x7F7F7F7Fu) ^ 0x7F7F7F7Fu;  // zero byte where the code is NaN
-      nan_bytes |= (y - 0x01010101u) & ~y & 0x80808080u;
-    }
-    uint32_t o[8];
-    if (nan_bytes == 0 && b != 255) {
-      const uint32_t e = b == 0 ? 0x0040u : (b << 7);  // BF16 2^(b-127) (2^-127 is subnormal)
-      const uint32_t scale2 = e | (e << 16);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          // [0, c_lo, 0, c_hi]: each E4M3 byte in the high byte of a 16-bit half
-          const uint32_t P = __byte_perm(wv[j], 0u, h == 0 ? 0x1404 : 0x3424);
-          const uint32_t bits = ((P >> 4) & 0x07F007F0u) | (P & 0x80008000u);
-          o[2 * j + h] = bf16x2_mul_rn(bf16x2_mul_rn(bits, 0x7B807B80u), scale2);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint16_t h0 = mxfp8_to_bf16((uint8_t)(wv[j]), b);
-        const uint16_t h1 = mxfp8_to_bf16((uint8_t)(wv[j] >> 8), b);
-        const uint16_t h2 = mxfp8_to_bf16((uint8_t)(wv[j] >> 16), b);
-        const uint16_t h3 = mxfp8_to_bf16((uint8_t)(wv[j] >> 24), b);
-        o[2 * j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-        o[2 * j + 1] = (uint32_t)h2 | ((uint32_t)h3 << 16);
+      for (int h = 0; h < 2; ++h) {
+        // [0, c_lo, 0, c_hi]: each E4M3 byte in the high byte of a 16-bit half
+        const uint32_t P = __byte_perm(wv[j], 0u, h == 0 ? 0x1404 : 0x3424);
+        const uint32_t bits = ((P >> 4) & 0x07F007F0u) | (P & 0x80008000u);
+        o[2 * j + h] = bf16x2_mul_rn(bf16x2_mul_rn(bits, 0x7B807B80u), scale2);
       }
     }
-    __stcs(out + 2 * i, make_uint4(o[0], o[1], o[2], o[3]));
-    __stcs(out + 2 * i + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint16_t h0 = mxfp8_to_bf16((uint8_t)(wv[j]), b);
+      const uint16_t h1 = mxfp8_to_bf16((uint8_t)(wv[j] >> 8), b);
+      const uint16_t h2 = mxfp8_to_bf16((uint8_t)(wv[j] >> 16), b);
+      const uint16_t h3 = mxfp8_to_bf16((uint8_t)(wv[j] >> 24), b);
+      o[2 * j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+      o[2 * j + 1] = (uint32_t)h2 | ((uint32_t)h3 << 16);
+    }
+  }
+  __stcs(out, make_uint4(o[0], o[1], o[2], o[3]));
+  __stcs(out + 1, make_uint4(o[4], o[5], o[6], o[7]));
+}
+
+// DU chunks per thread and iteration, all loaded before any is decoded.
+constexpr int DU = 4;
+
+__global__ void decode_mxfp8_kernel(const uint4* __restrict__ words, const uint8_t* __restrict__ sc,
+                                    int64_t chunks, uint4* __restrict__ out) {
+  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (int64_t base = 0; base + tid < chunks; base += DU * nthreads) {
+    uint4 w[DU];
+    uint32_t b[DU];
+#pragma unroll
+    for (int j = 0; j < DU; ++j) {
+      const int64_t i = base + j * nthreads + tid;
+      w[j] = make_uint4(0, 0, 0, 0);
+      b[j] = 0;
+      if (i < chunks) {
+        w[j] = __ldcs(words + i);
+        b[j] = sc[i >> 1];  // cols % 32 == 0: chunk i lies in scale block i / 2
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < DU; ++j) {
+      const int64_t i = base + j * nthreads + tid;
+      if (i < chunks) decode_chunk(w[j], b[j], out + 2 * i);
+    }
   }
 }
 
@@ -277,9 +299,10 @@ int launch_pack(int src_kind, const void* src, const void* aux0, const void* aux
 int launch_decode_mxfp8(const uint32_t* words, const uint8_t* scales, int64_t rows, int64_t cols,
                         uint16_t* out, const Exec& ex) {
   const int64_t chunks = rows * (cols / 16);
-  int64_t blocks = (chunks + 255) / 256;
-  const int64_t cap = (int64_t)ex.num_sms * 16;
+  int64_t blocks = (chunks / DU + 255) / 256;
+  const int64_t cap = (int64_t)ex.num_sms * 8;
   if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
   decode_mxfp8_kernel<<<(unsigned)blocks, 256, 0, ex.stream>>>((const uint4*)words, scales, chunks,
                                                                (uint4*)out);
   return cuda_status(cudaGetLastError());

@@ -157,6 +157,27 @@ def test_quantize_act_bit_exact(shape):
     assert np.array_equal(xs.cpu().numpy().view(np.uint32), as_ref.view(np.uint32))
 
 
+def test_quantize_act_bit_exact_wide_ranges():
+    """33 M values whose 64-groups span the whole BF16 exponent range (each
+    group scaled by its own power of two, some groups subnormal), against the
+    oracle's IEEE quotient and round-to-nearest-even."""
+    t, k = 4096, 8192
+    g = torch.Generator().manual_seed(1234)
+    x = torch.randn(t, k, generator=g)
+    e = torch.randint(-140, 120, (t, k // 64), generator=g).float()
+    x = (x.view(t, k // 64, 64) * torch.exp2(e)[..., None]).view(t, k)
+    x = x.to(torch.bfloat16)
+    qa_ref, as_ref = oracle.quantize_act(bits16(x))
+    xq = torch.empty(t, k, dtype=torch.int8, device=DEV)
+    xs = torch.empty(t, k // 64, dtype=torch.float32, device=DEV)
+    q.qlin_quantize_act(x.to(DEV), xq, xs)
+    torch.cuda.synchronize()
+    assert np.array_equal(xs.cpu().numpy().view(np.uint32), as_ref.view(np.uint32))
+    got = xq.cpu().numpy()
+    bad = np.argwhere(got != qa_ref)
+    assert bad.size == 0, (bad[:5], got[tuple(bad[0])], qa_ref[tuple(bad[0])])
+
+
 # ---------------------------------------------------------------------------
 # BF16-route GEMV
 # ---------------------------------------------------------------------------
