@@ -76,7 +76,16 @@ struct Cfg {
   static_assert(NS >= 2, "pipeline needs two stages");
   static_assert(NWG * WG_COLS <= (int)TMEM_COLS, "tensor memory budget");
   static constexpr size_t SMEM = (size_t)NS * L::STAGE + 1024 + 512;
+  static constexpr int RND = TP <= 32 ? TP : 32;      // accumulator columns per epilogue read
 };
+
+// Keeps uses of r after the preceding tcgen05.wait::ld (volatile asm statements
+// keep their order; plain arithmetic on r would not be tied to the wait).
+template <int W>
+__device__ __forceinline__ void after_wait(uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < W; ++i) asm volatile("" : "+r"(r[i]));
+}
 
 struct TcArgs {
   const void* scales;
@@ -126,7 +135,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1 + 32);  // TMA issue + 32 scale-copy arrivals
-      mbar_init(&empty[s], 1);      // released by the epilogue once the unit is done
+      mbar_init(&empty[s], 128);    // every epilogue thread, once done with the unit's scales
     }
     for (int i = 0; i < 2 * NWG; ++i) {
       mbar_init(&d_full[i], C::GB);  // one tcgen05.commit per issuing warp
@@ -343,14 +352,26 @@ __global__ void __launch_bounds__(THREADS, 1)
           float sc = 1.0f;
           if constexpr (Tr::PER_GROUP) sc = __half2float(sc_row[bi * GB + g]);
 #pragma unroll
-          for (int c = 0; c < TP; c += 16) {
-            if (c < T) {
-              uint32_t vr[16];
-              tmem_ld_x16(d_addr + g * TP + c, vr);
-              tmem_ld_wait();
-              tmem_fill_x16(d_addr + g * TP + c, 0u);  // ready for a later batch
+          for (int c0 = 0; c0 < TP; c0 += C::RND) {
+            if (c0 < T) {
+              // one round trip for up to RND columns, in 16-column loads (the
+              // last may run past T: those columns stay zero).  Narrower loads
+              // chosen at run time (x1..x8) measured twice as slow overall.
+              uint32_t vr[C::RND];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) acc[c + j] = fmaf(sc, __uint_as_float(vr[j]), acc[c + j]);
+              for (int c = 0; c < C::RND; c += 16)
+                if (c0 + c < T) tmem_ld_x16(d_addr + g * TP + c0 + c, vr + c);
+              tmem_ld_wait();
+              after_wait<C::RND>(vr);
+#pragma unroll
+              for (int c = 0; c < C::RND; c += 16) {
+                if (c0 + c < T) {
+                  tmem_fill_x16(d_addr + g * TP + c0 + c, 0u);  // ready for a later batch
+#pragma unroll
+                  for (int j = 0; j < 16; ++j)
+                    acc[c0 + c + j] = fmaf(sc, __uint_as_float(vr[c + j]), acc[c0 + c + j]);
+                }
+              }
             }
           }
         }
@@ -359,8 +380,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive(&d_empty[bw * 2 + ds]);
       }
       // every batch of the unit is done: the TMA stage (codes, activations,
-      // scales) can be refilled
-      if (!dead && et == 0) mbar_arrive(&empty[s]);
+      // scales) can be refilled once all four epilogue warps have read its scales
+      if (!dead) mbar_arrive(&empty[s]);
       ring.next(NS);
       const int cur_tile = tile;
       if (++ch == cpt) {
