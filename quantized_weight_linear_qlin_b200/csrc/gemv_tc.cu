@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (!dead) {
           tc_fence_after();
-#pragma unroll 1
+#pragma unroll 2
           for (int g = 0; g < GB; ++g) {
             const int gi = bi * GB + g;  // group within the unit
             uint32_t v[C::ACOLS];
