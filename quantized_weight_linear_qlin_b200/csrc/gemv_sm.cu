@@ -15,11 +15,13 @@
 //   warp 0      TMA: the unit's packed codes (two 128-byte-wide boxes), the Q5
 //               high-bit plane and the matching activation columns into a ring
 //               of shared-memory stages; its lanes cp.async the group scales;
-//   warps 1-8   thread = (weight row, half of the unit's groups): expand each
-//               group to exact BF16 pairs (the same exponent-bias tricks as the
-//               tensor-core kernel), FMA against x from shared memory into one
-//               FP32 sum per group, apply the group's FP16 scale; the two halves
-//               of a row meet by a shuffle at the end of the CTA's part of a tile.
+//   warps 1-16  thread = (weight row, quarter of the unit's groups; 8 rows per
+//               warp): expand each group to exact BF16 pairs (the same
+//               exponent-bias tricks as the tensor-core kernel), FMA against x
+//               from shared memory into one FP32 sum per group, apply the group's
+//               FP16 scale; the parts of a row meet by shuffles at the end of the
+//               CTA's part of a tile.  (BF16 weights, two groups per unit: halves,
+//               16 rows per warp, warps 1-8.)
 // Tiles split between two CTAs meet in the workspace exactly as in the
 // tensor-core kernel (same layout, same deterministic reduction order).
 #include "qlin_gemv_common.cuh"
@@ -29,8 +31,6 @@ namespace {
 using namespace gemv;
 
 constexpr int SM_SMEM_BUDGET = 212992;
-constexpr int NCW = 8;                   // compute warps
-constexpr int SM_THREADS = 32 * (1 + NCW);
 constexpr int UBS = 2;                   // 128-byte code boxes per unit
 
 template <int FMT, int T>
@@ -54,6 +54,14 @@ struct SmCfg {
   static_assert(NS >= 2, "pipeline needs two stages");
   static constexpr size_t SMEM = (size_t)NS * STAGE + 1024 + 256;
   static constexpr int ACOLS = Tr::GK / 2;            // BF16 pairs per group
+  // a row's groups are split over PARTS lanes of one warp (RPW rows per warp);
+  // 128 rows then take NCW compute warps: 16 warps (4 per scheduler) keep the
+  // shared-memory and FMA latencies hidden
+  static constexpr int PARTS = GPC >= 4 ? 4 : GPC;
+  static constexpr int RPW = 32 / PARTS;
+  static constexpr int NCW = 128 / RPW;
+  static constexpr int THREADS = 32 * (1 + NCW);
+  static constexpr int GPP = GPC / PARTS;             // groups per part
 };
 
 struct SmArgs {
@@ -78,13 +86,13 @@ __device__ __forceinline__ void halves(uint32_t v, uint16_t& lo, uint16_t& hi) {
 }
 
 template <int FMT, int T>
-__global__ void __launch_bounds__(SM_THREADS, 1)
+__global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
     gemv_sm_kernel(const __grid_constant__ CUtensorMap tm_codes,
                    const __grid_constant__ CUtensorMap tm_hib,
                    const __grid_constant__ CUtensorMap tm_x, SmArgs args) {
   using Tr = TcT<FMT>;
   using C = SmCfg<FMT, T>;
-  constexpr int NS = C::NS, GPC = C::GPC;
+  constexpr int NS = C::NS, GPC = C::GPC, NCW = C::NCW, RPW = C::RPW, GPP = C::GPP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(base + NS * C::STAGE);
@@ -170,10 +178,10 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
       }
     }
   } else {
-    // ---- compute warps: row r of the tile, half h of the unit's groups
+    // ---- compute warps: row r of the tile, part h of the unit's groups
     const int cw = warp - 1;
-    const int r = cw * 16 + (lane & 15);
-    const int h = lane >> 4;
+    const int r = cw * RPW + (lane % RPW);
+    const int h = lane / RPW;
     const int et = r;  // index of the row within the tile
     float acc[T];
 #pragma unroll
@@ -200,8 +208,8 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
         const uint8_t* xs = st + C::OFF_X;
         const __half* sc_row = (const __half*)(st + C::OFF_SC) + r * GPC;
 #pragma unroll 2
-        for (int gg = 0; gg < GPC / 2; ++gg) {
-          const int gi = h * (GPC / 2) + gg;  // group within the unit
+        for (int gg = 0; gg < GPP; ++gg) {
+          const int gi = h * GPP + gg;  // group within the unit
           uint32_t v[C::ACOLS];
           // high-bit plane rows are UBS * 32 bytes; dequant_group adds r * 32
           dequant_group<FMT>(st + (gi / Tr::GPB) * BOX_BYTES,
@@ -244,9 +252,11 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
         ++tile;
       }
       if (!seg_last) continue;
-      // ---- the CTA's part of this tile is complete: the two halves of each row meet
+      // ---- the CTA's part of this tile is complete: the parts of each row meet
 #pragma unroll
-      for (int t = 0; t < T; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 16);
+      for (int o = RPW; o < 32; o <<= 1)
+#pragma unroll
+        for (int t = 0; t < T; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
       float rs = 1.0f;
       if constexpr (FMT == QLIN_FP8_ROW) {
         if (row < args.n) rs = __bfloat162float(((const __nv_bfloat16*)args.scales)[row]);
@@ -327,7 +337,7 @@ int launch_t(const CUtensorMap& mc, const CUtensorMap& mh, const CUtensorMap& mx
   auto kern = gemv_sm_kernel<FMT, T>;
   const cudaError_t e = set_smem_once<gemv_sm_kernel<FMT, T>>((int)C::SMEM);
   if (e != cudaSuccess) return cuda_status(e);
-  kern<<<grid, SM_THREADS, C::SMEM, st>>>(mc, mh, mx, a);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(mc, mh, mx, a);
   return cuda_status(cudaGetLastError());
 }
 
