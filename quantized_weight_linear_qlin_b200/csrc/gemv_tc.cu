@@ -66,13 +66,20 @@ struct Cfg {
   using L = Layout<FMT, TP, UB>;
   static constexpr int GPC = L::GPC, KC = L::KC, NS = L::NS;
   static constexpr int ACOLS = Tr::GK / 2;            // tensor-memory columns of one group's A
-  static constexpr bool fits(int gb) { return NWG * (gb * ACOLS + 2 * gb * TP) <= (int)TMEM_COLS; }
-  // groups per batch: one barrier, one commit and one epilogue wait per batch
-  static constexpr int GB = (GPC % 4 == 0 && fits(4)) ? 4 : (GPC % 2 == 0 && fits(2)) ? 2 : 1;
+  static constexpr bool fits(int gb, int nd) { return NWG * (gb * ACOLS + nd * gb * TP) <= (int)TMEM_COLS; }
+  static constexpr int gb_for(int nd) {
+    return (GPC % 4 == 0 && fits(4, nd)) ? 4 : (GPC % 2 == 0 && fits(2, nd)) ? 2 : 1;
+  }
+  // groups per batch: one barrier, one commit and one epilogue wait per batch.
+  // Fixed costs per batch (tensor-memory round trips, the barrier, the MMA
+  // issue) favour large batches: one accumulator slot per warpgroup when that
+  // allows more groups per batch than two slots do.
+  static constexpr int NDW = gb_for(1) > gb_for(2) ? 1 : 2;  // accumulator slots per warpgroup
+  static constexpr int GB = gb_for(NDW);
   static constexpr int BPU = GPC / GB;                // batches per unit
   static constexpr int A_COLS = GB * ACOLS;           // a warpgroup's A slot
   static constexpr int D_COLS = GB * TP;              // one accumulator slot (a batch)
-  static constexpr int WG_COLS = A_COLS + 2 * D_COLS; // per warpgroup: A slot + two accumulator slots
+  static constexpr int WG_COLS = A_COLS + NDW * D_COLS; // per warpgroup: A slot + accumulator slots
   static_assert(NS >= 2, "pipeline needs two stages");
   static_assert(NWG * WG_COLS <= (int)TMEM_COLS, "tensor memory budget");
   static constexpr size_t SMEM = (size_t)NS * L::STAGE + 1024 + 512;
@@ -116,7 +123,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sc_s = hib_s + NS * L::HIB_BYTES;                // NS x SC_BYTES
   uint64_t* full = (uint64_t*)(sc_s + NS * L::SC_BYTES);
   uint64_t* empty = full + NS;
-  uint64_t* d_full = empty + NS;        // [NWG][2]
+  uint64_t* d_full = empty + NS;        // [NWG][2], slots 0..NDW-1 used
   uint64_t* d_empty = d_full + 2 * NWG; // [NWG][2]
   uint32_t* tmem_slot = (uint32_t*)(d_empty + 2 * NWG);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
     for (int w = 0; w < NWG; ++w)
 #pragma unroll 1
-      for (int c = 0; c < 2 * C::D_COLS; c += 16)
+      for (int c = 0; c < C::NDW * C::D_COLS; c += 16)
         tmem_fill_x16(tmem + lo + w * C::WG_COLS + C::A_COLS + c, 0u);
     tmem_st_wait();
   }
@@ -261,10 +268,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (bw != wg) continue;
         const int ds = dr.slot;
         if (!dead) {
-          // the accumulator slot was read and re-zeroed by the epilogue, and the
-          // previous batch's MMAs (which read the A slot) are complete
-          bool ok = mbar_wait(&d_empty[wg * 2 + ds], (uint32_t)(dr.phase ^ 1));
-          if (ok && prev_slot >= 0) ok = mbar_wait(&d_full[wg * 2 + prev_slot], (uint32_t)prev_phase);
+          // the previous batch's MMAs (which read the A slot) are complete; the
+          // accumulator slot is waited for only by the issuing threads, so that
+          // the expansion overlaps the epilogue's draining of it
+          bool ok = true;
+          if (prev_slot >= 0) ok = mbar_wait(&d_full[wg * 2 + prev_slot], (uint32_t)prev_phase);
           if (!__all_sync(0xffffffffu, ok)) {
             dead = true;
             abort_now();
@@ -289,7 +297,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         named_barrier_sync(1 + wg, 128);
         // warp q issues group q of the batch from lane 0: one thread issues an
         // MMA only every ~45-80 cycles, threads of different warps in parallel
-        if (quarter < GB && lane == 0 && !dead) {
+        bool go = quarter < GB && lane == 0 && !dead;
+        // the accumulator slot was read and re-zeroed by the epilogue (each
+        // issuing thread waits for every use of its warpgroup's slots in order)
+        if (go && !mbar_wait(&d_empty[wg * 2 + ds], (uint32_t)(dr.phase ^ 1))) {
+          go = false;
+          abort_now();
+        }
+        if (go) {
           tc_fence_after();
           const int g = quarter;
           const int kofs = (bi * GB + g) * Tr::GK;  // K offset of the group inside the unit
@@ -302,7 +317,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         prev_slot = ds;
         prev_phase = dr.phase;
-        dr.next(2);
+        dr.next(C::NDW);
       }
       ring.next(NS);
     }
@@ -338,7 +353,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int bi = 0; bi < BPU; ++bi, bw = (bw + 1 == NWG) ? 0 : bw + 1) {
         const int ds = dr[bw].slot;
         const uint32_t dph = (uint32_t)dr[bw].phase;
-        dr[bw].next(2);
+        dr[bw].next(C::NDW);
         if (dead) continue;
         if (!__all_sync(0xffffffffu, mbar_wait(&d_full[bw * 2 + ds], dph))) {
           dead = true;
