@@ -456,9 +456,12 @@ def measure_rows(ctx):
     rows["decode_mxfp8_5120x17408"] = {"ms": round(ms, 4), "GB/s": round(b / ms / 1e6, 1),
                                        "frac_hbm": round(b / ms / 1e6 / hbm, 3)}
     del words, sc, out
-    # Q8 group-32 GEMV 5120x5120 and FP8 row head 152064x5120
+    # Q8 group-32 GEMV 5120x5120, and the 152064x5120 output head as row-scaled
+    # FP8 and as Q8 group-32 across T = 1..64 (the pages' FP8-vs-Q8 head crossover)
+    head_ts = (1, 17, 33, 48, 64)
     for name, fmt, n, k, ts in (("gemv_q8_5120x5120", q.Q8_G32, 5120, 5120, T_LIST),
-                                ("gemv_fp8_head_152064x5120", q.FP8_ROW, 152064, 5120, (1, 33))):
+                                ("gemv_fp8_head_152064x5120", q.FP8_ROW, 152064, 5120, head_ts),
+                                ("gemv_q8_head_152064x5120", q.Q8_G32, 152064, 5120, head_ts)):
         pw = packed(q, synth, fmt, n, k, 3, dev)
         res = {}
         for t in ts:
@@ -470,6 +473,10 @@ def measure_rows(ctx):
             res[f"T={t}"] = {"us": round(ms * 1e3, 1), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
         rows[name] = res
         del pw
+    # which head format is faster at each T (time per call)
+    fp8h, q8h = rows["gemv_fp8_head_152064x5120"], rows["gemv_q8_head_152064x5120"]
+    rows["head_faster_format"] = {tk: ("fp8_row" if fp8h[tk]["us"] <= q8h[tk]["us"] else "q8_g32")
+                                  for tk in fp8h if tk in q8h}
     # headline matrices per T (kernel view)
     gu, dn = ctx["copies"][0]
     for name, pw in (("gemv_q4_gate_up", gu), ("gemv_q5_down", dn)):
@@ -665,7 +672,12 @@ def main():
     out, ctx = run_ours(args, dist)
     if dist.rank == 0:
         if not args.no_rows:
-            out["rows"] = measure_rows(ctx)
+            # the per-row measurements come after the headline; a failure there
+            # is reported in the line instead of losing it
+            try:
+                out["rows"] = measure_rows(ctx)
+            except Exception as e:  # pragma: no cover
+                out["rows"] = {"error": f"{type(e).__name__}: {e}"[:300]}
         out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
         print(json.dumps(out))
     dist.barrier()

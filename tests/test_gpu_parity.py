@@ -258,6 +258,9 @@ def test_gemv_bf16_weights_prefill_sizes(t):
     ("down_q5", q.Q5_G64, 5120, 17408, 33),
     ("q8_5120", q.Q8_G32, 5120, 5120, 17),
     ("head_fp8", q.FP8_ROW, 152064, 5120, 1),
+    # the head in both formats at the top of the verify range (FP8-vs-Q8 crossover)
+    ("head_q8_T64", q.Q8_G32, 152064, 5120, 64),
+    ("head_fp8_T64", q.FP8_ROW, 152064, 5120, 64),
 ])
 def test_gemv_full_size_sampled_rows(name, fmt, n, k, t):
     """Full-size weights in the bench's launch configuration; the oracle
