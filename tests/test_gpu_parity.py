@@ -408,3 +408,96 @@ def test_gemm_a8_full_size_sampled(name, fmt, n, k):
     torch.cuda.synchronize()
     got = y[toks.to(DEV)][:, rows.to(DEV)].cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - yr) <= 5e-6 * br)
+
+
+# ---------------------------------------------------------------------------
+# ties: quotients exactly on k + 1/2 (hand-worked groups, tests/golden)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,fmt", [("q4_group", "q4"), ("q5_group", "q5"), ("q8_group", "q8")])
+def test_pack_ties_bit_exact(golden, name, fmt):
+    ex = golden["ties"][name]
+    gs = 32 if fmt == "q8" else 64
+    w = torch.full((3, 4 * gs), float(ex["rest"]), dtype=torch.float32)
+    for r in range(3):
+        w[r, r * gs:r * gs + len(ex["w_head"])] = torch.tensor(ex["w_head"]) * (-1) ** r
+    ref = oracle.pack(FMTS[fmt], w.numpy())
+    pw = pack_gpu(FMTS[fmt], w.to(DEV))
+    torch.cuda.synchronize()
+    assert_packed_equal(pw, ref)
+
+
+@pytest.mark.parametrize("name", ["act_group_unit_scale", "act_group_half_scale"])
+def test_quantize_act_ties_bit_exact(golden, name):
+    ex = golden["ties"][name]
+    x = torch.full((2, 128), float(ex["rest"]), dtype=torch.float32)
+    x[0, :len(ex["x_head"])] = torch.tensor(ex["x_head"])
+    x[1, 64:64 + len(ex["x_head"])] = -torch.tensor(ex["x_head"])
+    x = x.to(torch.bfloat16)
+    qa_ref, as_ref = oracle.quantize_act(bits16(x))
+    assert list(qa_ref[0, :len(ex["codes_head"])]) == ex["codes_head"]
+    xq = torch.empty(2, 128, dtype=torch.int8, device=DEV)
+    xs = torch.empty(2, 2, dtype=torch.float32, device=DEV)
+    q.qlin_quantize_act(x.to(DEV), xq, xs)
+    torch.cuda.synchronize()
+    assert np.array_equal(xq.cpu().numpy(), qa_ref)
+    assert np.array_equal(xs.cpu().numpy().view(np.uint32), as_ref.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# one 27B-class layer's projections on the int8 route at the long-chunk
+# prefill sizes, and the decode MLP with the formats swapped
+# ---------------------------------------------------------------------------
+LAYER = [("q", 6144, 5120), ("k", 1024, 5120), ("v", 1024, 5120), ("o", 5120, 6144),
+         ("gate", 17408, 5120), ("up", 17408, 5120), ("down", 5120, 17408)]
+
+
+@pytest.mark.parametrize("t", [512, 1792, 8192])
+@pytest.mark.parametrize("variant", ["mixed", "all_q5"])
+@pytest.mark.parametrize("proj", [p[0] for p in LAYER])
+def test_gemm_a8_layer_sweep_sampled(proj, variant, t):
+    """Sampled rows and tokens, always including the last row tile and the
+    last token tile, at the int8 route's 5e-6 bound; the full output is
+    written (no on-chip wait may run out)."""
+    _, n, k = next(p for p in LAYER if p[0] == proj)
+    fmt = q.Q5_G64 if (variant == "all_q5" or proj == "down") else q.Q4_G64
+    w = synth.weights_f32(n, k, seed=synth.seed_for(4, 10 + LAYER.index((proj, n, k))), device=DEV)
+    x = synth.activations_bf16(t, k, seed=synth.seed_for(4, 30 + k % 97), device=DEV)
+    pw = pack_gpu(fmt, w, allow_a8=True)
+    y = torch.empty(t, n, dtype=torch.bfloat16, device=DEV)
+    ws = q.Workspace(DEV).ensure(q.qlin_gemm_a8_workspace_bytes(t, n, k))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q.qlin_gemm_a8(pw, y, x=x, y_dtype=q.OUT_BF16, workspace=ws, dev_status=status)
+    g = torch.Generator().manual_seed(n + t)
+    rows = torch.cat([torch.randperm(n, generator=g)[:10], torch.tensor([n - 128, n - 1])]).unique()
+    toks = torch.cat([torch.randperm(t, generator=g)[:8], torch.tensor([0, t - 128, t - 1])]).unique()
+    ref = oracle.pack(fmt, w[rows.to(DEV)].cpu().numpy())
+    qa, as_ = oracle.quantize_act(bits16(x[toks.to(DEV)]))
+    yr, br = oracle.gemm_a8(ref, qa, as_, nthreads=8)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    got = y[toks.to(DEV)][:, rows.to(DEV)].float().cpu().numpy().astype(np.float64)
+    bad = np.abs(got - yr) > 5e-6 * br + np.abs(yr) * 2.0 ** -8
+    assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
+    assert torch.isfinite(y.float()).all()
+
+
+@pytest.mark.parametrize("t", [1, 4, 17, 33])
+@pytest.mark.parametrize("name,fmt,n,k", [("gate_up_q5", q.Q5_G64, 34816, 5120),
+                                          ("down_q4", q.Q4_G64, 5120, 17408)])
+def test_gemv_decode_mlp_swapped_formats(name, fmt, n, k, t):
+    w = synth.weights_f32(n, k, seed=synth.seed_for(1, 40), device=DEV)
+    x = synth.activations_bf16(t, k, seed=synth.seed_for(1, 41), device=DEV)
+    pw = pack_gpu(fmt, w)
+    y = torch.empty(t, n, dtype=torch.bfloat16, device=DEV)
+    ws = q.Workspace(DEV).ensure(q.qlin_gemv_workspace_bytes(pw, t))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q.qlin_gemv(pw, x, y, q.OUT_BF16, workspace=ws, dev_status=status)
+    g = torch.Generator().manual_seed(t)
+    rows = torch.cat([torch.randperm(n, generator=g)[:40], torch.tensor([0, n - 1])]).unique()
+    ref = oracle.pack(fmt, w[rows.to(DEV)].cpu().numpy())
+    yr, br = oracle.gemv(ref, bits16(x), nthreads=8)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    got = y[:, rows.to(DEV)].float().cpu().numpy().astype(np.float64)
+    bad = np.abs(got - yr) > 1e-3 * br + np.abs(yr) * 2.0 ** -8
+    assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])

@@ -63,6 +63,35 @@ def test_golden_act_group(orc, golden):
     assert not qa[0, 3:].any()
 
 
+def _tie_row(ex, width):
+    v = np.full((1, width), ex["rest"], np.float32)
+    v[0, :len(ex["w_head"] if "w_head" in ex else ex["x_head"])] = ex["w_head"] if "w_head" in ex else ex["x_head"]
+    return v
+
+
+@pytest.mark.parametrize("name,fmt", [("q4_group", Q4), ("q5_group", Q5), ("q8_group", Q8)])
+def test_golden_pack_ties_round_half_even(orc, golden, name, fmt):
+    """w/s exactly on k + 1/2: the codes are the even neighbours (a
+    round-half-away-from-zero oracle fails here)."""
+    ex = golden["ties"][name]
+    pw = orc.pack(fmt, _tie_row(ex, GS[fmt]))
+    assert pw["scales"][0, 0] == int(ex["scale_f16"], 16)
+    s = _f16_val(pw["scales"][0, 0])
+    wdq = orc.dequant(pw)[0]
+    for i, q in enumerate(ex["codes_head"]):
+        assert wdq[i] == q * s, (i, wdq[i] / s, q)
+    assert not wdq[len(ex["codes_head"]):].any()
+
+
+@pytest.mark.parametrize("name", ["act_group_unit_scale", "act_group_half_scale"])
+def test_golden_act_ties_round_half_even(orc, golden, name):
+    ex = golden["ties"][name]
+    qa, as_ = orc.quantize_act(_bf16(_tie_row(ex, 64)))
+    assert as_[0, 0] == np.float32(ex["scale_f32"])
+    assert list(qa[0, :len(ex["codes_head"])]) == ex["codes_head"]
+    assert not qa[0, len(ex["codes_head"]):].any()
+
+
 def test_page_constants_used(orc, golden):
     c = golden["constants"]
     x = np.zeros((1, c["act_group"]["value"] * 2), np.float32)
