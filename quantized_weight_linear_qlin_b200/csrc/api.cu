@@ -19,6 +19,10 @@ int launch_gemv_sm(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
 size_t gemv_tc_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
 int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                    const Exec& ex);
+bool gemv_f16_supported(const qlin_weights& w, int64_t t);
+size_t gemv_f16_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
+int launch_gemv_f16(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
+                    const Exec& ex);
 
 namespace {
 
@@ -106,18 +110,29 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
   return r == CUDA_SUCCESS ? QLIN_OK : QLIN_ERR_CUDA;
 }
 
-// T <= 64 runs on the tensor cores; BF16 weights at prefill sizes (T > 64)
-// and Q5 rows whose high-bit plane is not 16-byte aligned per row use the
-// CUDA-core kernel.
-// BF16 weights at more than 64 tokens (the GDN a/b projection at prefill):
-// the tensor-core kernel in 64-token chunks, one after the other on the stream
-// (the weights, 1 MB for 96 x 5120, stay in L2 between chunks).
+// Kernel choice (measured on B200, calls queued, L2 flushed):
+//  - FP8-row weights, and Q8 group-32 matrices of at least 2^27 weights (the
+//    output head): gemv_f16 (group scale folded into an FP16 A operand, one
+//    accumulator per tile segment): E4M3 and Q8 expand in few instructions,
+//    and the fixed per-call costs are spread over many units;
+//  - Q4 / Q5 and the smaller Q8 matrices: T = 1 on the CUDA cores (gemv_sm),
+//    2 <= T <= 64 on gemv_tc (exact BF16 integer codes, one FP32 sum per
+//    group scaled in the epilogue): the nibble expansion of gemv_f16 costs
+//    about 13 instructions per 32-bit word, which made it slower there;
+//  - BF16 weights: gemv_tc, in 64-token chunks above 64 tokens (the GDN a/b
+//    projection at prefill; the weights, 1 MB for 96 x 5120, stay in L2);
+//  - rows that are not whole units: the CUDA-core kernel.
 constexpr int64_t kTcMaxT = 64;
 static bool bf16_chunked(const qlin_weights& w, int64_t t) {
   return w.fmt == QLIN_BF16 && t > kTcMaxT && gemv_tc_supported(w, kTcMaxT);
 }
+static bool use_f16(const qlin_weights& w, int64_t t) {
+  const bool wanted = w.fmt == QLIN_FP8_ROW || (w.fmt == QLIN_Q8_G32 && w.n * w.k >= ((int64_t)1 << 27));
+  return wanted && gemv_f16_supported(w, t);
+}
 
 size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
+  if (use_f16(w, t)) return gemv_f16_workspace_bytes(w, t, num_sms);
   if (gemv_sm_supported(w, t)) return gemv_sm_workspace_bytes(w, t, num_sms);
   if (bf16_chunked(w, t)) return gemv_tc_workspace_bytes(w, kTcMaxT, num_sms);
   if (gemv_tc_supported(w, t)) return gemv_tc_workspace_bytes(w, t, num_sms);
@@ -126,7 +141,7 @@ size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
 
 int launch_gemv(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                 const Exec& ex) {
-  // T = 1: CUDA-core kernel (mixed-precision FMA); T <= 64: tensor cores
+  if (use_f16(w, t)) return launch_gemv_f16(w, x, t, y, y_dtype, ex);
   if (gemv_sm_supported(w, t)) return launch_gemv_sm(w, x, t, y, y_dtype, ex);
   if (bf16_chunked(w, t)) {
     const size_t ysz = y_dtype == QLIN_OUT_F32 ? 4 : 2;

@@ -113,14 +113,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same test, but the thread may be suspended (up to `suspend_ns`) until the
+// phase completes instead of returning at once: waiting warps then take no
+// issue slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete.  Returns false when
 // the wait ran out (kWaitLimitNs) -- the caller then abandons its work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  unsigned long long t0 = global_ns();
+  const unsigned long long t0 = global_ns();
   while (true) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if (global_ns() - t0 > kWaitLimitNs) return false;
   }
 }
@@ -178,6 +190,16 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar))
       : "memory");
+}
+// True in exactly one lane of the (converged) warp.  Code around it stays
+// warp-uniform, so the operands of the single-thread tcgen05 instructions
+// (descriptors, tensor-memory addresses) can live in uniform registers.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(pred));
+  return pred != 0;
 }
 // Named barrier among `count` threads (whole warps).
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
@@ -349,6 +371,10 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t addr) {
 __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(m >> 4) << 24);
+}
+// Instruction descriptor: kind::f16 with FP16 A and B, F32 accumulator, K-major.
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 // Instruction descriptor: kind::f16 with BF16 A and B, F32 accumulator, K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {

@@ -501,3 +501,29 @@ def test_gemv_decode_mlp_swapped_formats(name, fmt, n, k, t):
     got = y[:, rows.to(DEV)].float().cpu().numpy().astype(np.float64)
     bad = np.abs(got - yr) > 1e-3 * br + np.abs(yr) * 2.0 ** -8
     assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
+
+
+def test_gemv_q8_head_overflowing_scales_exact_path():
+    """A Q8 group-32 matrix of 2^27 weights takes the kernel that folds the
+    FP16 group scale into an FP16 operand; rows whose scale is above 511.75
+    (q * s could overflow FP16) are recomputed exactly on the CUDA cores."""
+    n, k, t = 32768, 4096, 3
+    w = synth.weights_f32(n, k, seed=77, device=DEV)
+    huge = torch.tensor([5, 1000, 4097, n - 1], device=DEV)
+    w[huge] = w[huge] * 5e6  # |w| up to ~5e5: group scales ~4e3
+    x = synth.activations_bf16(t, k, seed=78, device=DEV)
+    pw = pack_gpu(q.Q8_G32, w)
+    y = torch.empty(t, n, dtype=torch.float32, device=DEV)
+    ws = q.Workspace(DEV).ensure(q.qlin_gemv_workspace_bytes(pw, t))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q.qlin_gemv(pw, x, y, q.OUT_F32, workspace=ws, dev_status=status)
+    rows = torch.cat([huge.cpu(), torch.tensor([0, 6, 999, 1001, 4096, n - 2])])
+    ref = oracle.pack(q.Q8_G32, w[rows.to(DEV)].cpu().numpy())
+    assert (oracle.dequant(ref)[:4] != 0).any()
+    yr, br = oracle.gemv(ref, bits16(x), nthreads=8)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    got = y[:, rows.to(DEV)].cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    bad = np.abs(got - yr) > 1e-3 * br
+    assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
