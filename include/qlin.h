@@ -94,6 +94,7 @@ extern "C" {
 #define QLIN_SRC_BF16 1        /* bfloat16[N][K]                                */
 #define QLIN_SRC_MXFP8 2       /* uint32 words[N][K/4] + uint8 UE8M0 [N][K/32]  */
 #define QLIN_SRC_MLX_AFFINE8 3 /* uint8 q[N][K] + f16 scale, f16 bias [N][K/128]*/
+#define QLIN_SRC_FP8_BLOCK128 4 /* E4M3 uint8[N][K] + float32 [ceil(N/128)][ceil(K/128)] */
 
 /* ---- output dtypes ------------------------------------------------------ */
 #define QLIN_OUT_BF16 0
@@ -140,6 +141,15 @@ QLIN_API int qlin_packed_bytes(int fmt, int64_t n, int64_t k, size_t* codes_byte
  *   MLX_AFFINE8  w = q * scale + bias as one FP32 fused multiply-add, rounded
  *         to BF16 [same page, step 2]; `src_aux0` = f16 scales, `src_aux1` =
  *         f16 biases, one per 128 columns.
+ *   FP8_BLOCK128  E4M3 codes uint8[N][K] with one float32 scale per 128 x 128
+ *         block (`src_aux0` = the weight_scale_inv grid, row-major
+ *         [ceil(N/128)][ceil(K/128)]): value = E4M3 * scale as one FP32
+ *         multiplication (exact when the scale has at most 20 significant
+ *         bits, e.g. a BF16 scale), rounded to BF16; an E4M3 NaN code gives
+ *         0x7FC0 with its sign ["...EfficientThink-Uncensored FP8 for NInfer",
+ *         "Conversion and verification": block-wise to per-row].  With
+ *         dst->fmt = FP8_ROW this is the page's re-encode to one BF16 scale
+ *         per row.
  * Then quantized: Q4/Q5/Q8: per (row, group) s = FP16_rne(amax / Qmax) with
  * Qmax = 7 / 15 / 127 and q = clamp(rint(w / s)) against the stored scale
  * (0 when s == 0).  FP8_ROW: sc = BF16_rne(rowmax|w| / 448), code =

@@ -44,13 +44,14 @@ def lib():
         L.oracle_pack_fp8_row.argtypes = [vp, i64, i64, vp, vp]
         L.oracle_decode_mxfp8.argtypes = [vp, vp, i64, i64, vp]
         L.oracle_decode_mlx_affine.argtypes = [vp, vp, vp, i64, i64, vp]
+        L.oracle_decode_fp8_block128.argtypes = [vp, vp, i64, i64, vp]
         L.oracle_dequant.argtypes = [i32, vp, vp, vp, i64, i64, vp]
         L.oracle_gemv.argtypes = [i32, vp, vp, vp, i64, i64, vp, i64, vp, vp, i32]
         L.oracle_quantize_act.argtypes = [vp, i64, i64, vp, vp]
         L.oracle_group_sums.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp]
         L.oracle_gemm_a8.argtypes = [i32, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, i32]
         for name in ("oracle_to_bf16", "oracle_pack_groupwise", "oracle_pack_fp8_row", "oracle_decode_mxfp8",
-                     "oracle_decode_mlx_affine", "oracle_dequant", "oracle_gemv",
+                     "oracle_decode_mlx_affine", "oracle_decode_fp8_block128", "oracle_dequant", "oracle_gemv",
                      "oracle_quantize_act", "oracle_group_sums", "oracle_gemm_a8"):
             getattr(L, name).restype = C.c_int
         _lib = L
@@ -157,6 +158,17 @@ def decode_mlx_affine(q, scales, biases, rows, cols):
     out = np.zeros((rows, cols), np.uint16)
     _check(lib().oracle_decode_mlx_affine(_p(q), _p(scales), _p(biases), rows, cols, _p(out)),
            "decode_mlx_affine")
+    return out
+
+
+def decode_fp8_block128(codes, scale_inv, rows, cols):
+    """E4M3 codes uint8[rows][cols] + float32 scale_inv[ceil(rows/128)][ceil(cols/128)]
+    -> bfloat16 bits [rows][cols]."""
+    codes = _c(codes, np.uint8)
+    scale_inv = _c(scale_inv, np.float32)
+    out = np.zeros((rows, cols), np.uint16)
+    _check(lib().oracle_decode_fp8_block128(_p(codes), _p(scale_inv), rows, cols, _p(out)),
+           "decode_fp8_block128")
     return out
 
 

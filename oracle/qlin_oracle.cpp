@@ -343,6 +343,38 @@ int oracle_decode_mxfp8(const uint32_t* words, const uint8_t* scales, int64_t ro
   return 0;
 }
 
+// ---- FP8 block-128 source decode -------------------------------------------
+// [ROWFP8] "Conversion and verification": the checkpoint stores a projection
+// as E4M3 codes with a weight_scale_inv value per 128x128 weight block; each
+// code is decoded in FP32 (E4M3 value times the block's scale) and the decoded
+// values are re-encoded (per row, fp8_row_maxabs, or into any other target).
+// Reading: the block grid is float32 [ceil(rows/128)][ceil(cols/128)]
+// row-major; value = float32(e4m3(code) * scale) with one IEEE rounding (exact
+// whenever the scale has at most 20 significant bits, e.g. a BF16 scale: the
+// page's "fits exactly"); the value is then taken to BF16 (RNE) like every
+// non-F32 source of this library, which is the page's "source value's own
+// BF16 rounding" in its error bound.  E4M3 NaN codes decode to the BF16 NaN
+// with their sign.
+// Pinned by: the exact product for BF16-representable scales (numpy float64),
+// a hand example, and the page's element bound after the row re-encode.
+int oracle_decode_fp8_block128(const uint8_t* codes, const float* scale_inv, int64_t rows,
+                               int64_t cols, uint16_t* out) {
+  int64_t gcols = (cols + 127) / 128;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < cols; ++c) {
+      uint8_t code = codes[r * cols + c];
+      double e = e4m3_value(code);
+      if (std::isnan(e)) {
+        out[r * cols + c] = (uint16_t)(((code & 0x80) ? 0x8000 : 0) | 0x7FC0);
+        continue;
+      }
+      float v = (float)e * scale_inv[(r / 128) * gcols + c / 128];  // one FP32 rounding
+      out[r * cols + c] = bf16_rne((double)v);
+    }
+  }
+  return 0;
+}
+
 // ---- MLX affine int8 decode -------------------------------------------------
 // [MXFP8] step 2: uint8 codes, per-128-group F16 scale and F16 bias,
 // w = q * scale + bias, decoded to BF16.  Reading: one FP32 fused

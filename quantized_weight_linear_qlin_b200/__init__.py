@@ -13,7 +13,7 @@ import torch
 
 __all__ = [
     "QlinError", "Q4_G64", "Q5_G64", "Q8_G32", "FP8_ROW", "BF16",
-    "SRC_F32", "SRC_BF16", "SRC_MXFP8", "SRC_MLX_AFFINE8", "OUT_BF16", "OUT_F32",
+    "SRC_F32", "SRC_BF16", "SRC_MXFP8", "SRC_MLX_AFFINE8", "SRC_FP8_BLOCK128", "OUT_BF16", "OUT_F32",
     "ALLOW_A8", "DEBUG_GROUP_SUMS", "PackedWeights", "Workspace", "lib",
     "qlin_packed_bytes", "qlin_pack_weights", "qlin_decode_mxfp8", "qlin_quantize_act",
     "qlin_gemv", "qlin_gemv_workspace_bytes", "qlin_gemm_a8", "qlin_gemm_a8_workspace_bytes",
@@ -21,7 +21,7 @@ __all__ = [
 ]
 
 Q4_G64, Q5_G64, Q8_G32, FP8_ROW, BF16 = 0, 1, 2, 3, 4
-SRC_F32, SRC_BF16, SRC_MXFP8, SRC_MLX_AFFINE8 = 0, 1, 2, 3
+SRC_F32, SRC_BF16, SRC_MXFP8, SRC_MLX_AFFINE8, SRC_FP8_BLOCK128 = 0, 1, 2, 3, 4
 OUT_BF16, OUT_F32 = 0, 1
 ALLOW_A8 = 0x1
 DEBUG_GROUP_SUMS = 0x1

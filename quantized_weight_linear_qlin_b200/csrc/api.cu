@@ -196,6 +196,9 @@ int qlin_pack_weights(int src_kind, const void* src, const void* src_aux0, const
       if (dst->k % 128 || !src_aux0 || !src_aux1 || !aligned16(src_aux0) || !aligned16(src_aux1))
         return QLIN_ERR_INVALID_ARG;
       break;
+    case QLIN_SRC_FP8_BLOCK128:
+      if (!src_aux0 || !aligned16(src_aux0)) return QLIN_ERR_INVALID_ARG;
+      break;
     default:
       return QLIN_ERR_INVALID_ARG;
   }

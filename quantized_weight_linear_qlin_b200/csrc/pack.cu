@@ -5,7 +5,8 @@
 //
 // Sources: "Qwen3.8-27B MXFP8-CRACK -- NInfer artifact", "How it was built"
 // (step 1 MXFP8, step 2 MLX affine int8); "Qwen3.8-27B EfficientThink-
-// Uncensored FP8 for NInfer", "Conversion and verification" (fp8_row_maxabs);
+// Uncensored FP8 for NInfer", "Conversion and verification" (E4M3 codes with a
+// weight_scale_inv per 128 x 128 block, re-encoded with fp8_row_maxabs);
 // "Qwen3.8-27B for NInfer -- RTX 5080 16 GB", "Quantization profile"
 // (Q4G64_F16S, Q5G64_F16S); "...NVFP4-NInferV3", "What is in the file" (Q8).
 #include "qlin_internal.cuh"
@@ -55,6 +56,14 @@ __device__ __forceinline__ float source_value(const Src& s, int64_t r, int64_t c
       uint8_t code = (uint8_t)(w >> (8 * (c & 3)));
       uint32_t b = ((const uint8_t*)s.aux0)[r * (s.k / 32) + c / 32];
       return bf16_bits_to_float(mxfp8_to_bf16(code, b));
+    }
+    case QLIN_SRC_FP8_BLOCK128: {
+      // E4M3 code times its 128 x 128 block's scale in FP32 (one rounding),
+      // then BF16; an E4M3 NaN code gives the BF16 NaN with its sign
+      const uint8_t code = ((const uint8_t*)s.src)[r * s.k + c];
+      if ((code & 0x7F) == 0x7F) return bf16_bits_to_float((uint16_t)(0x7FC0 | ((code & 0x80) << 8)));
+      const float sc = ((const float*)s.aux0)[(r >> 7) * ((s.k + 127) >> 7) + (c >> 7)];
+      return __bfloat162float(__float2bfloat16_rn(__fmul_rn(e4m3_to_float(code), sc)));
     }
     default: {  // MLX affine int8: one FP32 fma, then BF16
       uint8_t q = ((const uint8_t*)s.src)[r * s.k + c];

@@ -9,7 +9,8 @@ Distributions follow the workloads the pages describe for a 27B-class decoder
 (outlier rows); activations ~N(0, 1) in BF16 with 0.5% of the channels scaled
 by 20 for every token (outlier channels); MXFP8 sources with E4M3 codes of
 N(0, 1) and block exponents b uniform in [117, 127]; MLX affine int8 sources
-with uniform uint8 codes.  No dataset or checkpoint is involved.
+with uniform uint8 codes; block-wise FP8 sources with E4M3 codes of N(0, 1)
+and random power-of-two-ish block scales.  No dataset or checkpoint is involved.
 
 Generation runs on the requested torch device with a seeded torch.Generator;
 the same (seed, device type) always yields the same bytes.
@@ -62,6 +63,20 @@ def mxfp8_source(rows: int, cols: int, seed: int, device="cpu", b_lo=117, b_hi=1
     scales = torch.randint(b_lo, b_hi + 1, (rows, cols // 32), generator=g, device=device,
                            dtype=torch.int32).to(torch.uint8)
     return words, scales
+
+
+def fp8_block128_source(rows: int, cols: int, seed: int, device="cpu", log2_lo=-8.0, log2_hi=-4.0):
+    """(codes uint8[rows][cols] = E4M3 of N(0, 1) draws, no NaN; block scales
+    float32[ceil(rows/128)][ceil(cols/128)] = 2^u with u uniform in [log2_lo, log2_hi]).
+    The default range puts the decoded weights near N(0, 0.02) with blocks of
+    different magnitude, as in a block-wise FP8 checkpoint."""
+    g = _gen(seed, device)
+    v = torch.randn((rows, cols), generator=g, device=device, dtype=torch.float32)
+    codes = v.to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    gr, gc = (rows + 127) // 128, (cols + 127) // 128
+    u = torch.rand((gr, gc), generator=g, device=device, dtype=torch.float32)
+    scales = torch.exp2(log2_lo + (log2_hi - log2_lo) * u)
+    return codes, scales
 
 
 def mlx_affine_source(rows: int, cols: int, seed: int, device="cpu"):

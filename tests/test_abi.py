@@ -112,6 +112,11 @@ def test_host_validation_rejects_before_cuda(L):
     w64 = _weights(q.Q4_G64, 4, 64)
     assert L.qlin_pack_weights(q.SRC_MLX_AFFINE8, fake, fake, fake, C.byref(w64),
                                C.byref(ex)) == q.ERR_INVALID_ARG
+    # block-128 FP8 source needs its scale grid, 16-byte aligned
+    assert L.qlin_pack_weights(q.SRC_FP8_BLOCK128, fake, None, None, C.byref(w64),
+                               C.byref(ex)) == q.ERR_INVALID_ARG
+    assert L.qlin_pack_weights(q.SRC_FP8_BLOCK128, fake, odd, None, C.byref(w64),
+                               C.byref(ex)) == q.ERR_INVALID_ARG
 
 
 def test_product_path_has_no_cpu_fallback():

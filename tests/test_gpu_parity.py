@@ -527,3 +527,42 @@ def test_gemv_q8_head_overflowing_scales_exact_path():
     assert np.isfinite(got).all()
     bad = np.abs(got - yr) > 1e-3 * br
     assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
+
+
+# ---------------------------------------------------------------------------
+# FP8 block-128 source (E4M3 + weight_scale_inv per 128 x 128 block) -> any
+# target; FP8_ROW is the block -> row re-encode
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("fmt", list(FMTS))
+@pytest.mark.parametrize("shape", [(200, 320), (384, 1024)])
+def test_pack_from_fp8_block128_bit_exact(fmt, shape):
+    rows, cols = shape
+    codes, sc = synth.fp8_block128_source(rows, cols, seed=31 + rows)
+    sc = sc.clone()
+    sc[0, 0] = 0.0  # an all-zero block
+    dec = oracle.decode_fp8_block128(codes.numpy(), sc.numpy(), rows, cols)
+    ref = oracle.pack(FMTS[fmt], bf16_value(dec).astype(np.float32))
+    pw = q.PackedWeights(FMTS[fmt], rows, cols, device=DEV)
+    q.qlin_pack_weights(q.SRC_FP8_BLOCK128, codes.to(DEV), pw, aux0=sc.to(DEV))
+    torch.cuda.synchronize()
+    assert_packed_equal(pw, ref)
+
+
+def test_pack_from_fp8_block128_full_size_rows_bit_exact():
+    """A 17408 x 5120 text projection re-encoded from block-128 to row FP8;
+    sampled rows (every row band of 128, first and last) against the oracle."""
+    rows, cols = 17408, 5120
+    codes, sc = synth.fp8_block128_source(rows, cols, seed=synth.seed_for(2, 5), device=DEV)
+    pw = q.PackedWeights(q.FP8_ROW, rows, cols, device=DEV)
+    q.qlin_pack_weights(q.SRC_FP8_BLOCK128, codes, pw, aux0=sc)
+    sel = torch.cat([torch.arange(0, rows, 131), torch.tensor([rows - 1])])
+    bands = (sel // 128).unique()
+    sc_sub = sc.cpu().numpy()
+    dec = np.concatenate([oracle.decode_fp8_block128(codes[int(r)].cpu().numpy()[None, :],
+                                                     sc_sub[int(r) // 128][None, :], 1, cols) for r in sel])
+    ref = oracle.pack(q.FP8_ROW, bf16_value(dec).astype(np.float32))
+    torch.cuda.synchronize()
+    got = gpu_packed_to_numpy(pw)
+    assert np.array_equal(got["codes"][sel.numpy()], ref["codes"])
+    assert np.array_equal(got["scales"][sel.numpy()], ref["scales"])
+    assert len(bands) > 100

@@ -353,3 +353,100 @@ def test_gemm_a8_scaled_matches_group_sums(orc):
         # and the int8 route approximates the BF16 route within the quantization noise
         yb, bb = orc.gemv(pw, x)
         assert np.all(np.abs(y - yb) <= 0.05 * bb)
+
+
+# ---- FP8 block-128 source (E4M3 codes + weight_scale_inv per 128x128 block) ----
+def _e4m3_vals(codes):
+    """E4M3 code -> float64 through torch's own float8_e4m3fn conversion."""
+    return torch.from_numpy(np.asarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _bf16_bits_of_f32(v32):
+    return torch.from_numpy(np.asarray(v32, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_golden_fp8_block128(orc, golden):
+    ex = golden["fp8_block128"]
+    codes = np.full((2, 128), int(ex["rest_code"], 16), np.uint8)
+    codes[0, :4] = [int(c, 16) for c in ex["codes_head"]]
+    out = orc.decode_fp8_block128(codes, np.array([[ex["block_scale"]]], np.float32), 2, 128)
+    assert [int(v) for v in out[0, :4]] == [int(b, 16) for b in ex["bf16_head"]]
+    assert not out[0, 4:].any() and not out[1].any()
+    pw = orc.pack(FP8, _bf16_val(out[:1]))
+    assert pw["scales"][0] == int(ex["row_scale_bf16"], 16)
+    assert [int(c) for c in pw["codes"][0, :4]] == [int(c, 16) for c in ex["codes_head"]]
+
+
+def _block_source(rng, rows, cols, bf16_scales):
+    codes = rng.integers(0, 256, (rows, cols)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C  # no NaN codes
+    gr, gc = (rows + 127) // 128, (cols + 127) // 128
+    sc = np.exp2(rng.uniform(-14, -4, (gr, gc))).astype(np.float32) * rng.uniform(1, 2, (gr, gc)).astype(np.float32)
+    if bf16_scales:
+        sc = _bf16_val(_bf16_bits_of_f32(sc)).astype(np.float32)
+    return codes, sc
+
+
+def test_fp8_block128_exact_for_bf16_scales(orc):
+    """A BF16 block scale times an E4M3 value has at most 12 significant bits:
+    the FP32 product is exact (the page's "fits exactly") and the decode is
+    that exact value rounded once to BF16.  Ragged grid: 200 x 300."""
+    rng = np.random.default_rng(21)
+    rows, cols = 200, 300
+    codes, sc = _block_source(rng, rows, cols, True)
+    full = np.repeat(np.repeat(sc.astype(np.float64), 128, 0), 128, 1)[:rows, :cols]
+    exact = _e4m3_vals(codes) * full
+    assert np.array_equal(exact.astype(np.float32).astype(np.float64), exact)  # exact in FP32
+    out = orc.decode_fp8_block128(codes, sc, rows, cols)
+    assert np.array_equal(out, _bf16_bits_of_f32(exact.astype(np.float32)))
+
+
+def test_fp8_block128_general_fp32_scales(orc):
+    """Scales with a full FP32 mantissa: one IEEE single product (numpy float32)
+    then BF16 rounding (torch)."""
+    rng = np.random.default_rng(22)
+    rows, cols = 131, 256
+    codes, sc = _block_source(rng, rows, cols, False)
+    full = np.repeat(np.repeat(sc, 128, 0), 128, 1)[:rows, :cols]
+    prod = _e4m3_vals(codes).astype(np.float32) * full  # IEEE single multiply
+    out = orc.decode_fp8_block128(codes, sc, rows, cols)
+    assert np.array_equal(out, _bf16_bits_of_f32(prod))
+
+
+def test_fp8_block128_to_row_within_page_bound(orc):
+    """The page's verification bound for the block -> row re-encode: every
+    element stays within the E4M3 half-ulp of its own magnitude at the stored
+    row scale plus the source value's own BF16 rounding."""
+    rng = np.random.default_rng(23)
+    rows, cols = 256, 384
+    codes, sc = _block_source(rng, rows, cols, False)
+    full = np.repeat(np.repeat(sc.astype(np.float64), 128, 0), 128, 1)[:rows, :cols]
+    src = (_e4m3_vals(codes).astype(np.float32) * full.astype(np.float32)).astype(np.float64)
+    dec = orc.decode_fp8_block128(codes, sc, rows, cols)
+    pw = orc.pack(FP8, _bf16_val(dec))
+    rs = _bf16_val(pw["scales"]).astype(np.float64)[:, None]
+    got = orc.dequant(pw)
+    mag = np.abs(src) / rs
+    e = np.floor(np.log2(np.maximum(mag, 2.0 ** -6)))
+    half_ulp = np.exp2(np.maximum(e, -6) - 3) / 2 * rs  # E4M3: 3 mantissa bits, min normal 2^-6
+    bf16_err = np.abs(_bf16_val(dec).astype(np.float64) - src)
+    assert np.all(np.abs(got - src) <= half_ulp + bf16_err + 1e-300)
+
+
+def test_fp8_block128_row_reencode_is_identity_when_scales_agree(orc):
+    """A row whose codes all share one BF16 block scale and which holds a
+    +-448 code re-encodes to the very same codes, with the block scale as its
+    row scale (the page's bit-exact re-encode of the converter's arithmetic)."""
+    rng = np.random.default_rng(24)
+    rows, cols = 64, 128
+    codes, _ = _block_source(rng, rows, cols, True)
+    codes[:, 5] = np.where(rng.integers(0, 2, rows) > 0, 0x7E, 0xFE)
+    sc = np.array([[2.0 ** -7 * 1.5]], np.float32)
+    dec = orc.decode_fp8_block128(codes, sc, rows, cols)
+    pw = orc.pack(FP8, _bf16_val(dec))
+    assert np.all(_bf16_val(pw["scales"]) == sc[0, 0])
+    ref = codes.copy()
+    ref[(ref & 0x7F) == 0] = 0x00  # -0 and +0 both encode +0 after the round trip
+    got = pw["codes"].copy()
+    got[(got & 0x7F) == 0] = 0x00
+    assert np.array_equal(got, ref)
