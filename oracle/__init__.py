@@ -50,9 +50,12 @@ def lib():
         L.oracle_quantize_act.argtypes = [vp, i64, i64, vp, vp]
         L.oracle_group_sums.argtypes = [i32, vp, vp, vp, i64, i64, i64, vp]
         L.oracle_gemm_a8.argtypes = [i32, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, i32]
+        L.oracle_quantize_act_fp8.argtypes = [vp, i64, i64, vp, vp]
+        L.oracle_gemm_fp8.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, i32]
         for name in ("oracle_to_bf16", "oracle_pack_groupwise", "oracle_pack_fp8_row", "oracle_decode_mxfp8",
                      "oracle_decode_mlx_affine", "oracle_decode_fp8_block128", "oracle_dequant", "oracle_gemv",
-                     "oracle_quantize_act", "oracle_group_sums", "oracle_gemm_a8"):
+                     "oracle_quantize_act", "oracle_group_sums", "oracle_gemm_a8",
+                     "oracle_quantize_act_fp8", "oracle_gemm_fp8"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -212,6 +215,30 @@ def gemm_a8(pw, qa, as_, nthreads=1, with_bound=True):
     b = np.zeros((t, n), np.float64) if with_bound else None
     _check(lib().oracle_gemm_a8(pw["fmt"], _p(pw["codes"]), _p(pw["hibits"]), _p(pw["scales"]),
                                 _p(qa), _p(as_), t, n, k, _p(y), _p(b), int(nthreads)), "gemm_a8")
+    return y, b
+
+
+def quantize_act_fp8(x_bf16):
+    """Per-token E4M3 activations: (xq uint8[t][k], xs float32[t])."""
+    x = _c(x_bf16, np.uint16)
+    t, k = x.shape
+    xq = np.zeros((t, k), np.uint8)
+    xs = np.zeros((t,), np.float32)
+    _check(lib().oracle_quantize_act_fp8(_p(x), t, k, _p(xq), _p(xs)), "quantize_act_fp8")
+    return xq, xs
+
+
+def gemm_fp8(pw, xq, xs, nthreads=1, with_bound=True):
+    """Row-FP8 weights (oracle.pack(FP8_ROW, ...)) x per-token FP8 activations."""
+    assert pw["fmt"] == FP8_ROW
+    xq = _c(xq, np.uint8)
+    xs = _c(xs, np.float32)
+    t = xq.shape[0]
+    n, k = pw["n"], pw["k"]
+    y = np.zeros((t, n), np.float64)
+    b = np.zeros((t, n), np.float64) if with_bound else None
+    _check(lib().oracle_gemm_fp8(_p(pw["codes"]), _p(pw["scales"]), _p(xq), _p(xs), t, n, k, _p(y), _p(b),
+                                 int(nthreads)), "gemm_fp8")
     return y, b
 
 

@@ -525,4 +525,59 @@ int oracle_gemm_a8(int fmt, const void* codes, const void* hibits, const uint16_
   return 0;
 }
 
+// ---- FP8-activation route: per-token E4M3 activations --------------------
+// [ROWFP8] "Conversion and verification", "Hardware fit": the row-scaled FP8
+// weights run on FP8-activation tensor-core routes.  The page fixes no
+// activation scheme; reading, mirroring fp8_row_maxabs on the activation side:
+// per token t, a = max_k |x[t][k]| (exact in FP32), xs = a / 448 (FP32, kept
+// FP32), xq = (xs == 0) ? 0x00 : E4M3_rne_satfinite(x / xs) (FP32 quotient).
+// Pinned by: hand examples (incl. a tie), the amax element at +-448, zero
+// tokens, and the E4M3 half-ulp bound of every element.
+int oracle_quantize_act_fp8(const uint16_t* x, int64_t t, int64_t k, uint8_t* xq, float* xs) {
+  for (int64_t tt = 0; tt < t; ++tt) {
+    const uint16_t* xr = x + tt * k;
+    float a = 0.0f;
+    for (int64_t i = 0; i < k; ++i) {
+      float m = std::fabs((float)bf16_value(xr[i]));
+      if (m > a) a = m;
+    }
+    float s = a / 448.0f;
+    xs[tt] = s;
+    for (int64_t i = 0; i < k; ++i)
+      xq[tt * k + i] = s == 0.0f ? (uint8_t)0 : e4m3_rne_satfinite((double)((float)bf16_value(xr[i]) / s));
+  }
+  return 0;
+}
+
+// ---- FP8-activation route: row-FP8 weights x per-token FP8 activations ------
+// y[t][n] = c * S with S = sum_k e4m3(wq[n][k]) * e4m3(xq[t][k]) (exact, in
+// double) and c = FP32(ws[n] * xs[t]), ws the BF16 row scale; reported in
+// double.  bound[t][n] = sum_k |e4m3(wq) ws| * |e4m3(xq) xs| (tolerance scale).
+// Pinned by: integer-valued E4M3 codes with unit scales equal an exact integer
+// matrix product.
+int oracle_gemm_fp8(const uint8_t* wq, const uint16_t* ws, const uint8_t* xq, const float* xs,
+                    int64_t t, int64_t n, int64_t k, double* y, double* bound, int nthreads) {
+  std::vector<double> xv((size_t)(t * k));
+  for (int64_t i = 0; i < t * k; ++i) xv[i] = e4m3_value(xq[i]);
+  parallel_rows(n, nthreads, [&](int64_t r0, int64_t r1) {
+    std::vector<double> wr((size_t)k);
+    for (int64_t r = r0; r < r1; ++r) {
+      for (int64_t e = 0; e < k; ++e) wr[e] = e4m3_value(wq[r * k + e]);
+      float wsr = (float)bf16_value(ws[r]);
+      for (int64_t tt = 0; tt < t; ++tt) {
+        double S = 0.0, A = 0.0;
+        const double* xr = xv.data() + tt * k;
+        for (int64_t e = 0; e < k; ++e) {
+          S += wr[e] * xr[e];
+          A += std::fabs(wr[e]) * std::fabs(xr[e]);
+        }
+        float c = wsr * xs[tt];
+        y[tt * n + r] = (double)c * S;
+        if (bound) bound[tt * n + r] = std::fabs((double)wsr * (double)xs[tt]) * A;
+      }
+    }
+  });
+  return 0;
+}
+
 }  // extern "C"

@@ -450,3 +450,55 @@ def test_fp8_block128_row_reencode_is_identity_when_scales_agree(orc):
     got = pw["codes"].copy()
     got[(got & 0x7F) == 0] = 0x00
     assert np.array_equal(got, ref)
+
+
+# ---- FP8-activation route ------------------------------------------------------
+def test_golden_fp8_act_token(orc, golden):
+    ex = golden["fp8_act_token"]
+    x = np.zeros((1, 64), np.float32)
+    x[0, :len(ex["x_head"])] = ex["x_head"]
+    xq, xs = orc.quantize_act_fp8(_bf16(x))
+    assert xs[0] == np.float32(ex["scale_f32"])
+    assert [int(c) for c in xq[0, :len(ex["codes_head"])]] == [int(c, 16) for c in ex["codes_head"]]
+    assert not xq[0, len(ex["codes_head"]):].any()
+
+
+def test_fp8_act_invariants(orc):
+    """amax element -> +-448 code; zero token -> scale 0, codes 0; every element
+    within half an E4M3 step of its own magnitude (scaled back by xs)."""
+    rng = np.random.default_rng(31)
+    t, k = 9, 1536
+    x = rng.standard_normal((t, k)).astype(np.float32) * np.exp2(rng.integers(-20, 20, (t, 1)))
+    x[3] = 0.0
+    xb = _bf16(x)
+    xf = _bf16_val(xb).astype(np.float64)
+    xq, xs = orc.quantize_act_fp8(xb)
+    assert xs[3] == 0 and not xq[3].any()
+    vals = _e4m3_vals(xq)
+    for tt in range(t):
+        if tt == 3:
+            continue
+        assert xs[tt] == np.float32(np.float32(np.abs(xf[tt]).max()) / np.float32(448.0))
+        i = int(np.argmax(np.abs(xf[tt])))
+        assert abs(vals[tt, i]) == 448.0
+        mag = np.abs(xf[tt]) / xs[tt]
+        e = np.floor(np.log2(np.maximum(mag, 2.0 ** -6)))
+        half = np.exp2(np.maximum(e, -6) - 3) / 2
+        assert np.all(np.abs(vals[tt] - xf[tt] / xs[tt]) <= half * (1 + 2.0 ** -20) + 2.0 ** -30)
+
+
+def test_gemm_fp8_reduces_to_integer_matmul(orc):
+    """Integer-valued E4M3 codes (|v| <= 16 are all exact) with unit scales:
+    the route is an exact integer matrix product."""
+    rng = np.random.default_rng(32)
+    n, k, t = 19, 320, 7
+    wi = rng.integers(-16, 17, (n, k))
+    xi = rng.integers(-16, 17, (t, k))
+    wi[:, 0] = 448 // 28 * 0  # keep the row max well inside
+    enc = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    pw = {"fmt": FP8, "n": n, "k": k, "codes": enc(wi), "hibits": None,
+          "scales": np.full((n,), 0x3F80, np.uint16)}
+    y, b = orc.gemm_fp8(pw, enc(xi), np.ones((t,), np.float32))
+    exact = (xi.astype(np.int64) @ wi.T.astype(np.int64)).astype(np.float64)
+    assert np.array_equal(y, exact)
+    assert np.array_equal(b, (np.abs(xi) @ np.abs(wi).T).astype(np.float64))
