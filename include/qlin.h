@@ -210,6 +210,34 @@ QLIN_API int qlin_gemm_a8(const qlin_weights* w, const uint16_t* x_bf16, const i
                  int64_t t, void* y, int y_dtype, uint32_t flags, int32_t* group_sums_dbg,
                  const qlin_exec* ex);
 
+/* Per-token FP8 activation quantization of x bfloat16[T][K] for the
+ * FP8-activation route: xs[t] = max_k |x[t][k]| / 448 (FP32, IEEE division)
+ * and xq[t][k] = E4M3(x / xs) rounded to nearest even with saturation to
+ * +-448 (all zero when xs == 0).  xq uint8[T][K] (E4M3 bytes), xs
+ * float32[T].  K % 16 == 0.  ["Qwen3.8-27B EfficientThink-Uncensored FP8 for
+ * NInfer", "Conversion and verification" and "Hardware fit": row-scaled FP8
+ * weights run on FP8-activation tensor-core routes; the page fixes no
+ * activation scheme, and one FP32 scale per token mirrors fp8_row_maxabs on
+ * the activation side.]  Bit-exact. */
+QLIN_API int qlin_quantize_act_fp8(const uint16_t* x_bf16, int64_t t, int64_t k, uint8_t* xq, float* xs,
+                                   const qlin_exec* ex);
+
+/* Workspace bytes qlin_gemm_fp8 needs when it quantizes T x K activations itself. */
+QLIN_API int qlin_gemm_fp8_workspace_bytes(int64_t t, int64_t k, size_t* bytes);
+
+/* FP8-activation projection (prefill and decode) for FP8_ROW weights
+ * (QLIN_ERR_UNSUPPORTED for any other format), any T >= 1.  Activations
+ * either as x_bf16 (qlin_quantize_act_fp8 runs inside the call into the
+ * workspace, xq/xs must be NULL) or pre-quantized as xq uint8[T][K] +
+ * xs float32[T] (x_bf16 NULL; no workspace needed).
+ * y[t][n] = FP32(ws[n] * xs[t]) * sum_k E4M3(w[n][k]) * E4M3(xq[t][k]),
+ * the products exact and the sum accumulated in FP32 on the tensor cores.
+ * Accuracy: |y - y_ref| <= 1e-5 * |ws xs| sum_k |w||xq| per element before
+ * the BF16 output rounding, y_ref the exact product of the same codes.
+ * [Same page, "Hardware fit".] */
+QLIN_API int qlin_gemm_fp8(const qlin_weights* w, const uint16_t* x_bf16, const uint8_t* xq, const float* xs,
+                           int64_t t, void* y, int y_dtype, const qlin_exec* ex);
+
 /* qlin_gemv without a caller workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory when they
  * call (memory planned once at start-up; plain C code owning only w, x and y).

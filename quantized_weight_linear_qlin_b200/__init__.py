@@ -17,7 +17,8 @@ __all__ = [
     "ALLOW_A8", "DEBUG_GROUP_SUMS", "PackedWeights", "Workspace", "lib",
     "qlin_packed_bytes", "qlin_pack_weights", "qlin_decode_mxfp8", "qlin_quantize_act",
     "qlin_gemv", "qlin_gemv_workspace_bytes", "qlin_gemm_a8", "qlin_gemm_a8_workspace_bytes",
-    "qlin_status_string", "qlin_gemv_noalloc",
+    "qlin_status_string", "qlin_gemv_noalloc", "qlin_quantize_act_fp8",
+    "qlin_gemm_fp8_workspace_bytes", "qlin_gemm_fp8",
 ]
 
 Q4_G64, Q5_G64, Q8_G32, FP8_ROW, BF16 = 0, 1, 2, 3, 4
@@ -34,6 +35,7 @@ EXPORTED = (
     "qlin_status_string", "qlin_packed_bytes", "qlin_pack_weights", "qlin_decode_mxfp8",
     "qlin_quantize_act", "qlin_gemv_workspace_bytes", "qlin_gemv",
     "qlin_gemm_a8_workspace_bytes", "qlin_gemm_a8", "qlin_gemv_noalloc",
+    "qlin_quantize_act_fp8", "qlin_gemm_fp8_workspace_bytes", "qlin_gemm_fp8",
 )
 
 
@@ -77,6 +79,9 @@ def lib():
         L.qlin_gemm_a8_workspace_bytes.argtypes = [i64, i64, i64, vp]
         L.qlin_gemm_a8.argtypes = [C.POINTER(_Weights), vp, vp, vp, i64, vp, i32, u32, vp,
                                    C.POINTER(_Exec)]
+        L.qlin_quantize_act_fp8.argtypes = [vp, i64, i64, vp, vp, C.POINTER(_Exec)]
+        L.qlin_gemm_fp8_workspace_bytes.argtypes = [i64, i64, vp]
+        L.qlin_gemm_fp8.argtypes = [C.POINTER(_Weights), vp, vp, vp, i64, vp, i32, C.POINTER(_Exec)]
         for name in EXPORTED[1:]:
             getattr(L, name).restype = i32
         _lib = L
@@ -238,4 +243,28 @@ def qlin_gemm_a8(w: PackedWeights, y, x=None, xq=None, xs=None, y_dtype=OUT_BF16
     e = _exec(stream, workspace, dev_status)
     _check(lib().qlin_gemm_a8(C.byref(d), _ptr(x), _ptr(xq), _ptr(xs), t, _ptr(y), y_dtype, flags,
                               _ptr(sums_dbg), C.byref(e)), "qlin_gemm_a8")
+    return y
+
+
+def qlin_quantize_act_fp8(x, xq, xs, stream=None):
+    t, k = x.shape
+    e = _exec(stream)
+    _check(lib().qlin_quantize_act_fp8(_ptr(x), t, k, _ptr(xq), _ptr(xs), C.byref(e)),
+           "qlin_quantize_act_fp8")
+    return xq, xs
+
+
+def qlin_gemm_fp8_workspace_bytes(t, k):
+    b = C.c_size_t()
+    _check(lib().qlin_gemm_fp8_workspace_bytes(t, k, C.byref(b)), "qlin_gemm_fp8_workspace_bytes")
+    return b.value
+
+
+def qlin_gemm_fp8(w: PackedWeights, y, x=None, xq=None, xs=None, y_dtype=OUT_BF16, workspace=None,
+                  stream=None, dev_status=None):
+    t = (x if x is not None else xq).shape[0]
+    d = w.desc()
+    e = _exec(stream, workspace, dev_status)
+    _check(lib().qlin_gemm_fp8(C.byref(d), _ptr(x), _ptr(xq), _ptr(xs), t, _ptr(y), y_dtype,
+                               C.byref(e)), "qlin_gemm_fp8")
     return y

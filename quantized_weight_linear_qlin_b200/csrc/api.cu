@@ -283,4 +283,43 @@ int qlin_gemm_a8(const qlin_weights* w, const uint16_t* x_bf16, const int8_t* xq
   return launch_gemm_a8(*w, x_bf16, xq, xs, t, y, y_dtype, flags, group_sums_dbg, e);
 }
 
+int qlin_quantize_act_fp8(const uint16_t* x_bf16, int64_t t, int64_t k, uint8_t* xq, float* xs,
+                          const qlin_exec* ex) {
+  if (!x_bf16 || !xq || !xs || t <= 0 || k <= 0 || k % 16) return QLIN_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(xq) || !aligned16(xs)) return QLIN_ERR_INVALID_ARG;
+  if (t > (int64_t)INT32_MAX) return QLIN_ERR_UNSUPPORTED;
+  Exec e;
+  int rc = make_exec(ex, &e);
+  if (rc) return rc;
+  return launch_quantize_act_fp8(x_bf16, t, k, xq, xs, e);
+}
+
+int qlin_gemm_fp8_workspace_bytes(int64_t t, int64_t k, size_t* bytes) {
+  if (!bytes || t <= 0 || k <= 0 || k % 16) return QLIN_ERR_INVALID_ARG;
+  *bytes = gemm_fp8_workspace_bytes(t, k);
+  return QLIN_OK;
+}
+
+int qlin_gemm_fp8(const qlin_weights* w, const uint16_t* x_bf16, const uint8_t* xq, const float* xs,
+                  int64_t t, void* y, int y_dtype, const qlin_exec* ex) {
+  int rc = check_weights(w);
+  if (rc) return rc;
+  if (w->fmt != QLIN_FP8_ROW) return QLIN_ERR_UNSUPPORTED;
+  if (t <= 0 || !y || !aligned16(y)) return QLIN_ERR_INVALID_ARG;
+  if (y_dtype != QLIN_OUT_BF16 && y_dtype != QLIN_OUT_F32) return QLIN_ERR_INVALID_ARG;
+  const bool fused = x_bf16 != nullptr;
+  if (fused == (xq != nullptr || xs != nullptr)) return QLIN_ERR_INVALID_ARG;
+  if (fused && !aligned16(x_bf16)) return QLIN_ERR_INVALID_ARG;
+  if (!fused && (!xq || !xs || !aligned16(xq) || !aligned16(xs))) return QLIN_ERR_INVALID_ARG;
+  if (t > (int64_t)INT32_MAX || w->n > (int64_t)INT32_MAX || w->k > (int64_t)INT32_MAX)
+    return QLIN_ERR_UNSUPPORTED;
+  Exec e;
+  if ((rc = make_exec(ex, &e))) return rc;
+  if (fused) {
+    const size_t need = gemm_fp8_workspace_bytes(t, w->k);
+    if (need > e.workspace_bytes || !e.workspace) return QLIN_ERR_WORKSPACE;
+  }
+  return launch_gemm_fp8(*w, x_bf16, xq, xs, t, y, y_dtype, e);
+}
+
 }  // extern "C"

@@ -118,6 +118,27 @@ def test_host_validation_rejects_before_cuda(L):
     assert L.qlin_pack_weights(q.SRC_FP8_BLOCK128, fake, odd, None, C.byref(w64),
                                C.byref(ex)) == q.ERR_INVALID_ARG
 
+    # FP8-activation route: FP8_ROW weights only, one activation form, K % 16
+    w8 = _weights(q.FP8_ROW, 256, 512)
+    assert L.qlin_gemm_fp8(C.byref(w), fake, None, None, 4, fake, q.OUT_BF16,
+                           C.byref(ex)) == q.ERR_UNSUPPORTED
+    assert L.qlin_gemm_fp8(C.byref(w8), fake, fake, fake, 4, fake, q.OUT_BF16,
+                           C.byref(ex)) == q.ERR_INVALID_ARG
+    assert L.qlin_gemm_fp8(C.byref(w8), None, fake, None, 4, fake, q.OUT_BF16,
+                           C.byref(ex)) == q.ERR_INVALID_ARG
+    assert L.qlin_gemm_fp8(C.byref(w8), None, fake, odd, 4, fake, q.OUT_BF16,
+                           C.byref(ex)) == q.ERR_INVALID_ARG
+    assert L.qlin_gemm_fp8(C.byref(w8), fake, None, None, 0, fake, q.OUT_BF16,
+                           C.byref(ex)) == q.ERR_INVALID_ARG
+    assert L.qlin_gemm_fp8(C.byref(w8), fake, None, None, 4, fake, 5,
+                           C.byref(ex)) == q.ERR_INVALID_ARG
+    assert L.qlin_quantize_act_fp8(fake, 4, 40, fake, fake, C.byref(ex)) == q.ERR_INVALID_ARG
+    assert L.qlin_quantize_act_fp8(fake, 4, 48, fake, odd, C.byref(ex)) == q.ERR_INVALID_ARG
+    b = C.c_size_t()
+    assert L.qlin_gemm_fp8_workspace_bytes(3, 40, C.byref(b)) == q.ERR_INVALID_ARG
+    assert L.qlin_gemm_fp8_workspace_bytes(3, 4096, C.byref(b)) == q.OK
+    assert b.value == (3 * 4096 + 255) // 256 * 256 + 3 * 4
+
 
 def test_product_path_has_no_cpu_fallback():
     """The binding refuses CPU tensors instead of computing on the host."""
