@@ -182,7 +182,10 @@ QLIN_API int qlin_gemv_workspace_bytes(const qlin_weights* w, int64_t t, size_t*
  * (QLIN_ERR_UNSUPPORTED above); BF16 weights: any T >= 1.  FP32 accumulation;
  * y_dtype QLIN_OUT_BF16 (RNE) or QLIN_OUT_F32.  The workspace must hold
  * qlin_gemv_workspace_bytes() and be zero-filled before its first use with
- * this library; every call leaves its counters at zero again.
+ * this library; every call that completes leaves its counters at zero again.
+ * After a call that reported QLIN_ERR_TIMEOUT its split-tile counters may be
+ * left non-zero: zero-fill the workspace again before its next use
+ * (qlin_gemv_noalloc clears its own counters on every call).
  * Accuracy: |y - y_ref| <= 1e-3 * sum_k |w||x| per element (plus the BF16
  * output rounding).  ["NInfer int8-prefill artifact for the RTX 4090",
  * "What changes": decode keeps the BF16 route; "...NVFP4-NInferV3", "How it
@@ -245,9 +248,13 @@ QLIN_API int qlin_gemm_fp8(const qlin_weights* w, const uint16_t* x_bf16, const 
  * cudaStream_t or NULL, dev_status as qlin_exec.dev_status, may be NULL); the
  * scratch qlin_gemv would take from qlin_exec.workspace comes instead from a
  * fixed 16 MiB device array inside the library, one per device.
+ * Argument errors are reported exactly as qlin_gemv reports them, before
+ * anything is enqueued (quantized weights with T > 64: QLIN_ERR_UNSUPPORTED).
  * Requests whose qlin_gemv_workspace_bytes() exceeds 16 MiB return
- * QLIN_ERR_WORKSPACE (T <= 64 on the quantized formats always fits; BF16
- * weights at large T * N may not).
+ * QLIN_ERR_WORKSPACE.  The tensor-core kernels need at most a few MiB at
+ * T <= 64; a matrix whose K is not a whole number of the kernels' column
+ * units (and is above 2048) runs on the CUDA-core kernel, which needs
+ * T * N * 4 bytes: e.g. Q4 152064 x 5184 at T = 64 needs 39 MB and is refused.
  * The first call on a device resolves the array's address and zero-fills it
  * (synchronously); make that first call before any stream capture.  Each call
  * clears the array's split-tile counters on `stream` before its kernels.

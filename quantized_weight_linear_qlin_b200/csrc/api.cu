@@ -2,6 +2,7 @@
 // dispatch to the kernel launchers.  Nothing here allocates device memory.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "qlin_internal.cuh"
@@ -31,18 +32,51 @@ std::once_flag g_encode_once;
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// SM count per device, queried once (0 = not yet known).
+std::atomic<int> g_num_sms[64];
+
 int make_exec(const qlin_exec* e, Exec* out) {
   out->stream = e ? (cudaStream_t)e->stream : (cudaStream_t)0;
   out->dev_status = e ? e->dev_status : nullptr;
   out->workspace = e ? e->workspace : nullptr;
   out->workspace_bytes = e ? e->workspace_bytes : 0;
+  if (out->workspace && !aligned16(out->workspace)) return QLIN_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QLIN_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&out->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return QLIN_ERR_CUDA;
-  if (out->workspace && !aligned16(out->workspace)) return QLIN_ERR_INVALID_ARG;
+  const bool cacheable = dev >= 0 && dev < 64;
+  int sms = cacheable ? g_num_sms[dev].load(std::memory_order_relaxed) : 0;
+  if (sms <= 0) {
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return QLIN_ERR_CUDA;
+    if (cacheable) g_num_sms[dev].store(sms, std::memory_order_relaxed);
+  }
+  out->num_sms = sms;
   return QLIN_OK;
 }
+
+// Encoded tensor maps of recent calls, per host thread: a decode loop calls
+// the same few projections over and over, and an encode costs about a
+// microsecond of driver time.  The key is every argument of the encode; a
+// cached map is only reused for the identical request.
+struct TmapKey {
+  const void* base;
+  uint64_t inner, outer, stride;
+  uint32_t box_inner, box_outer;
+  int dtype, swizzle;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && inner == o.inner && outer == o.outer && stride == o.stride &&
+           box_inner == o.box_inner && box_outer == o.box_outer && dtype == o.dtype &&
+           swizzle == o.swizzle;
+  }
+};
+constexpr int kTmapCache = 32;
+struct TmapCache {
+  TmapKey key[kTmapCache];
+  CUtensorMap map[kTmapCache];
+  bool used[kTmapCache] = {};
+  int next = 0;
+};
+thread_local TmapCache t_tmaps;
 
 int group_of(int fmt) {
   switch (fmt) {
@@ -100,6 +134,13 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
       g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
   });
   if (!g_encode) return QLIN_ERR_CUDA;
+  const TmapKey key{base, inner, outer, row_stride_bytes, box_inner, box_outer, (int)dtype, (int)swizzle};
+  TmapCache& c = t_tmaps;
+  for (int i = 0; i < kTmapCache; ++i)
+    if (c.used[i] && c.key[i] == key) {
+      *map = c.map[i];
+      return QLIN_OK;
+    }
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
@@ -107,7 +148,13 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
   CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? QLIN_OK : QLIN_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return QLIN_ERR_CUDA;
+  const int slot = c.next;
+  c.next = (c.next + 1) % kTmapCache;
+  c.key[slot] = key;
+  c.map[slot] = *map;
+  c.used[slot] = true;
+  return QLIN_OK;
 }
 
 // Kernel choice (measured on B200, calls queued, L2 flushed):
@@ -154,6 +201,18 @@ int launch_gemv(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, in
   }
   if (gemv_tc_supported(w, t)) return launch_gemv_tc(w, x, t, y, y_dtype, ex);
   return launch_gemv_cc(w, x, t, y, y_dtype, ex, (float*)ex.workspace);
+}
+
+// Host checks of qlin_gemv's arguments (shared with qlin_gemv_noalloc, which
+// must reject a call before it enqueues anything).
+int check_gemv_args(const qlin_weights* w, const uint16_t* x_bf16, int64_t t, const void* y,
+                    int y_dtype) {
+  int rc = check_weights(w);
+  if (rc) return rc;
+  if (!x_bf16 || !y || t <= 0 || !aligned16(x_bf16) || !aligned16(y)) return QLIN_ERR_INVALID_ARG;
+  if (y_dtype != QLIN_OUT_BF16 && y_dtype != QLIN_OUT_F32) return QLIN_ERR_INVALID_ARG;
+  if (w->fmt != QLIN_BF16 && t > 64) return QLIN_ERR_UNSUPPORTED;
+  return QLIN_OK;
 }
 
 }  // namespace qlin
@@ -239,11 +298,8 @@ int qlin_gemv_workspace_bytes(const qlin_weights* w, int64_t t, size_t* bytes) {
 
 int qlin_gemv(const qlin_weights* w, const uint16_t* x_bf16, int64_t t, void* y, int y_dtype,
               const qlin_exec* ex) {
-  int rc = check_weights(w);
+  int rc = qlin::check_gemv_args(w, x_bf16, t, y, y_dtype);
   if (rc) return rc;
-  if (!x_bf16 || !y || t <= 0 || !aligned16(x_bf16) || !aligned16(y)) return QLIN_ERR_INVALID_ARG;
-  if (y_dtype != QLIN_OUT_BF16 && y_dtype != QLIN_OUT_F32) return QLIN_ERR_INVALID_ARG;
-  if (w->fmt != QLIN_BF16 && t > 64) return QLIN_ERR_UNSUPPORTED;
   Exec e;
   if ((rc = make_exec(ex, &e))) return rc;
   size_t need = gemv_workspace_bytes(*w, t, e.num_sms);

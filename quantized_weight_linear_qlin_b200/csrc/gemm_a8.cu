@@ -577,7 +577,12 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
   cudaError_t e;
   auto kern = w.fmt == QLIN_Q4_G64 ? (debug ? gemm_a8_kernel<4, true> : gemm_a8_kernel<4, false>)
                                     : (debug ? gemm_a8_kernel<5, true> : gemm_a8_kernel<5, false>);
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = w.fmt == QLIN_Q4_G64
+          ? (debug ? set_smem_once<gemm_a8_kernel<4, true>>((int)smem)
+                   : set_smem_once<gemm_a8_kernel<4, false>>((int)smem))
+          : (debug ? set_smem_once<gemm_a8_kernel<5, true>>((int)smem)
+                   : set_smem_once<gemm_a8_kernel<5, false>>((int)smem));
+  if (e != cudaSuccess) return cuda_status(e);
   e = cudaLaunchKernelEx(&cfg, kern, tm_codes, tm_hib, tm_act, args);
   return cuda_status(e);
 }

@@ -212,8 +212,10 @@ int launch_cc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int 
   const int64_t kr = cc_krange(w.k);
   const int64_t ksplit = (w.k + kr - 1) / kr;
   dim3 grid((unsigned)((w.n + kRowsPerCta - 1) / kRowsPerCta), (unsigned)ksplit);
+  // at most kTokBlock x kMaxKRange floats (32 KB): within the default 48 KB of
+  // dynamic shared memory, so no attribute call is needed
+  static_assert(kTokBlock * kMaxKRange * sizeof(float) <= 48 * 1024, "staged x exceeds 48 KB");
   size_t smem = (size_t)kTokBlock * kr * sizeof(float);
-  cudaFuncSetAttribute(gemv_cc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (ksplit > 1) {
     cudaError_t e = cudaMemsetAsync(acc_ws, 0, (size_t)t * w.n * sizeof(float), ex.stream);
     if (e != cudaSuccess) return QLIN_ERR_CUDA;

@@ -53,9 +53,11 @@ void* scratch_for(int dev) {
 
 extern "C" QLIN_API int qlin_gemv_noalloc(const qlin_weights* w, const uint16_t* x_bf16, int64_t t,
                                           void* y, int y_dtype, void* stream, int32_t* dev_status) {
-  if (w == nullptr) return QLIN_ERR_INVALID_ARG;
+  // every argument check of qlin_gemv first: a rejected call enqueues nothing
+  int rc = qlin::check_gemv_args(w, x_bf16, t, y, y_dtype);
+  if (rc != QLIN_OK) return rc;
   size_t need = 0;
-  int rc = qlin_gemv_workspace_bytes(w, t, &need);
+  rc = qlin_gemv_workspace_bytes(w, t, &need);
   if (rc != QLIN_OK) return rc;
   if (need > qlin::kNoAllocBytes) return QLIN_ERR_WORKSPACE;  // larger than the fixed array
   int dev = -1;

@@ -41,6 +41,8 @@ size_t gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, int num_sms);
 int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, const float* xs,
                    int64_t t, void* y, int y_dtype, uint32_t flags, int32_t* sums_dbg,
                    const Exec& ex);
+int check_gemv_args(const qlin_weights* w, const uint16_t* x_bf16, int64_t t, const void* y,
+                    int y_dtype);
 size_t gemm_fp8_workspace_bytes(int64_t t, int64_t k);
 int launch_quantize_act_fp8(const uint16_t* x, int64_t t, int64_t k, uint8_t* xq, float* xs,
                             const Exec& ex);

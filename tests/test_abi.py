@@ -75,6 +75,10 @@ def test_host_validation_rejects_before_cuda(L):
     w = _weights(q.Q4_G64, 256, 512, flags=q.ALLOW_A8)
     # gemv: T above 64 is unsupported for quantized weights
     assert L.qlin_gemv(C.byref(w), fake, 65, fake, q.OUT_BF16, C.byref(ex)) == q.ERR_UNSUPPORTED
+    # the no-alloc variant runs the same checks first (before any CUDA call)
+    assert L.qlin_gemv_noalloc(C.byref(w), fake, 65, fake, q.OUT_BF16, None, None) == q.ERR_UNSUPPORTED
+    assert L.qlin_gemv_noalloc(C.byref(w), odd, 1, fake, q.OUT_BF16, None, None) == q.ERR_INVALID_ARG
+    assert L.qlin_gemv_noalloc(None, fake, 1, fake, q.OUT_BF16, None, None) == q.ERR_INVALID_ARG
     # misaligned activation / output pointers
     assert L.qlin_gemv(C.byref(w), odd, 1, fake, q.OUT_BF16, C.byref(ex)) == q.ERR_INVALID_ARG
     assert L.qlin_gemv(C.byref(w), fake, 1, odd, q.OUT_BF16, C.byref(ex)) == q.ERR_INVALID_ARG

@@ -58,3 +58,31 @@ def test_noalloc_rejects_requests_beyond_the_array():
     with pytest.raises(q.QlinError) as e:
         q.qlin_gemv_noalloc(pw, x, y, q.OUT_BF16)
     assert e.value.status == q.ERR_WORKSPACE
+
+
+def test_noalloc_reports_argument_errors_like_qlin_gemv():
+    """Quantized weights at T = 65: QLIN_ERR_UNSUPPORTED (as qlin_gemv), not a
+    workspace error, and nothing is enqueued."""
+    n, k, t = 34816, 5120, 65
+    pw = q.PackedWeights(q.Q4_G64, n, k, device=DEV)
+    x = torch.zeros(t, k, dtype=torch.bfloat16, device=DEV)
+    y = torch.empty(t, n, dtype=torch.bfloat16, device=DEV)
+    for call in (lambda: q.qlin_gemv_noalloc(pw, x, y, q.OUT_BF16),
+                 lambda: q.qlin_gemv(pw, x, y, q.OUT_BF16, workspace=q.Workspace(DEV))):
+        with pytest.raises(q.QlinError) as e:
+            call()
+        assert e.value.status == q.ERR_UNSUPPORTED
+
+
+def test_noalloc_rejects_quantized_cuda_core_shape_beyond_the_array():
+    """Q4 with K = 5184 (not a whole number of tensor-core column units) runs on
+    the CUDA-core kernel, whose split-K accumulator needs T * N * 4 = 39 MB at
+    N = 152064, T = 64: above the 16 MiB array."""
+    n, k, t = 152064, 5184, 64
+    pw = q.PackedWeights(q.Q4_G64, n, k, device=DEV)
+    assert q.qlin_gemv_workspace_bytes(pw, t) == t * n * 4
+    x = torch.zeros(t, k, dtype=torch.bfloat16, device=DEV)
+    y = torch.empty(t, n, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_gemv_noalloc(pw, x, y, q.OUT_BF16)
+    assert e.value.status == q.ERR_WORKSPACE
