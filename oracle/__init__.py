@@ -16,7 +16,7 @@ import numpy as np
 
 from . import build as _build
 
-Q4_G64, Q5_G64, Q8_G32, FP8_ROW, BF16 = 0, 1, 2, 3, 4
+Q4_G64, Q5_G64, Q8_G32, FP8_ROW, BF16, Q3_G64, Q6_G64 = 0, 1, 2, 3, 4, 5, 6
 
 _lib = None
 
@@ -106,6 +106,10 @@ def packed_shapes(fmt, n, k):
         return np.uint8, (n, k // 2), None, np.uint16, (n, k // 64)
     if fmt == Q5_G64:
         return np.uint8, (n, k // 2), (n, k // 8), np.uint16, (n, k // 64)
+    if fmt == Q3_G64:
+        return np.uint8, (n, k // 4), (n, k // 8), np.uint16, (n, k // 64)
+    if fmt == Q6_G64:
+        return np.uint8, (n, k // 2), (n, k // 4), np.uint16, (n, k // 64)
     if fmt == Q8_G32:
         return np.int8, (n, k), None, np.uint16, (n, k // 32)
     if fmt == FP8_ROW:
@@ -126,7 +130,7 @@ def pack(fmt, w):
     if fmt == FP8_ROW:
         scales = np.zeros(sshape, sdt)
         _check(lib().oracle_pack_fp8_row(_p(w), n, k, _p(codes), _p(scales)), "pack_fp8_row")
-    elif fmt in (Q4_G64, Q5_G64, Q8_G32):
+    elif fmt in (Q4_G64, Q5_G64, Q8_G32, Q3_G64, Q6_G64):
         scales = np.zeros(sshape, sdt)
         _check(lib().oracle_pack_groupwise(fmt, _p(w), n, k, _p(codes), _p(hib), _p(scales)),
                "pack_groupwise")

@@ -18,7 +18,8 @@
 //   [NVFP4] "Qwen3.8-27B-NVIDIA-NVFP4-NInferV3", "What is in the file" and
 //           "How it was created" (grouped Q4/Q5/Q8 with FP16 scales; head op).
 //   [RTX5080] "Qwen3.8-27B for NInfer -- RTX 5080 16 GB", "Quantization
-//           profile" (Q4G64_F16S, Q5G64_F16S).
+//           profile" (Q3G64_F16S, Q4G64_F16S, Q5G64_F16S).
+//   [MXFP8] "Caveats" also names Q6 among the groupwise formats.
 //   [A8]    "Qwen3.8-27B, NInfer int8-prefill artifact for the RTX 4090",
 //           "What changes" (the int8 prefill route).
 //
@@ -143,9 +144,22 @@ float clampf(float v, float lo, float hi) { return std::fmin(std::fmax(v, lo), h
 // Q8_G32: int8 two's complement codes, row-major.  FP8_ROW: E4M3 bytes,
 // row-major, one bfloat16 scale per row.  Scales of Q4/Q5 are binary16
 // [N][K/64]; of Q8 binary16 [N][K/32].
+// Two-bit ("crumb") plane, per row K/4 bytes read as K/16 little-endian
+// words.  Word c holds elements 16c..16c+15: element 16c+2s+o (s = 0..7,
+// o = 0..1) in bits [16o+2s, 16o+2s+2).
+// Q3_G64: u = q + 4 in [0, 7]; the crumb plane holds bits 0..1 of u (codes,
+// K/4 bytes per row) and a bit plane laid out as Q5's holds bit 2 (K/8 bytes
+// per row).  Q6_G64: u = q + 32 in [0, 63]; a nibble plane laid out as Q4's
+// holds bits 0..3 (codes, K/2 bytes per row) and a crumb plane holds bits
+// 4..5 (K/4 bytes per row).  Scales binary16 [N][K/64].
 // ---------------------------------------------------------------------------
 
-enum { FMT_Q4_G64 = 0, FMT_Q5_G64 = 1, FMT_Q8_G32 = 2, FMT_FP8_ROW = 3, FMT_BF16 = 4 };
+enum { FMT_Q4_G64 = 0, FMT_Q5_G64 = 1, FMT_Q8_G32 = 2, FMT_FP8_ROW = 3, FMT_BF16 = 4,
+       FMT_Q3_G64 = 5, FMT_Q6_G64 = 6 };
+
+inline bool is_groupwise64(int fmt) {
+  return fmt == FMT_Q4_G64 || fmt == FMT_Q5_G64 || fmt == FMT_Q3_G64 || fmt == FMT_Q6_G64;
+}
 
 inline uint32_t load_u32_le(const uint8_t* p) {
   return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
@@ -167,23 +181,44 @@ inline int hibit_bit(int64_t e) {  // bit position of element e's high bit
   return 16 * (i & 1) + 4 * jj + (i >> 1);
 }
 
-// Offset code u of element (row r, col e) of a Q4/Q5 matrix.
-int read_u(int bits, const uint8_t* codes, const uint8_t* hibits, int64_t k, int64_t r, int64_t e) {
-  const uint8_t* row = codes + r * (k / 2);
-  uint32_t w = load_u32_le(row + (e / 8) * 4);
-  int u = (int)((w >> nibble_bit(e)) & 0xF);
-  if (bits == 5) {
-    const uint8_t* hrow = hibits + r * (k / 8);
-    uint32_t h = load_u32_le(hrow + (e / 32) * 4);
-    u |= (int)((h >> hibit_bit(e)) & 1u) << 4;
+inline int crumb_bit(int64_t e) {  // bit position of element e inside its crumb word
+  int i = (int)(e & 15);
+  return 16 * (i & 1) + 2 * (i >> 1);
+}
+
+// Field readers of the planes (row r of a K-column matrix, element e).
+int nibble_at(const uint8_t* plane, int64_t k, int64_t r, int64_t e) {
+  uint32_t w = load_u32_le(plane + r * (k / 2) + (e / 8) * 4);
+  return (int)((w >> nibble_bit(e)) & 0xF);
+}
+int crumb_at(const uint8_t* plane, int64_t k, int64_t r, int64_t e) {
+  uint32_t w = load_u32_le(plane + r * (k / 4) + (e / 16) * 4);
+  return (int)((w >> crumb_bit(e)) & 0x3);
+}
+int bit_at(const uint8_t* plane, int64_t k, int64_t r, int64_t e) {
+  uint32_t h = load_u32_le(plane + r * (k / 8) + (e / 32) * 4);
+  return (int)((h >> hibit_bit(e)) & 1u);
+}
+
+// Offset code u of element (row r, col e) of a Q3/Q4/Q5/Q6 matrix.
+int read_u(int fmt, const uint8_t* codes, const uint8_t* hibits, int64_t k, int64_t r, int64_t e) {
+  switch (fmt) {
+    case FMT_Q4_G64: return nibble_at(codes, k, r, e);
+    case FMT_Q5_G64: return nibble_at(codes, k, r, e) | (bit_at(hibits, k, r, e) << 4);
+    case FMT_Q3_G64: return crumb_at(codes, k, r, e) | (bit_at(hibits, k, r, e) << 2);
+    default: return nibble_at(codes, k, r, e) | (crumb_at(hibits, k, r, e) << 4);  // Q6
   }
-  return u;
+}
+
+// Offset of u: 2^(bits - 1).
+int code_offset(int fmt) {
+  return fmt == FMT_Q4_G64 ? 8 : fmt == FMT_Q5_G64 ? 16 : fmt == FMT_Q3_G64 ? 4 : 32;
 }
 
 // Integer weight code q of any integer format.
 int weight_code(int fmt, const void* codes, const void* hibits, int64_t k, int64_t r, int64_t e) {
-  if (fmt == FMT_Q4_G64) return read_u(4, (const uint8_t*)codes, nullptr, k, r, e) - 8;
-  if (fmt == FMT_Q5_G64) return read_u(5, (const uint8_t*)codes, (const uint8_t*)hibits, k, r, e) - 16;
+  if (is_groupwise64(fmt))
+    return read_u(fmt, (const uint8_t*)codes, (const uint8_t*)hibits, k, r, e) - code_offset(fmt);
   return (int)((const int8_t*)codes)[r * k + e];  // Q8_G32
 }
 
@@ -238,22 +273,27 @@ int oracle_to_bf16(const float* v, int64_t count, uint16_t* out) {
 
 // ---- groupwise integer packing --------------------------------------------
 // [NVFP4] "What is in the file": Q4/Q5/Q8 grouped, FP16 scales.
-// [RTX5080] "Quantization profile": Q4G64_F16S, Q5G64_F16S (group 64).
+// [RTX5080] "Quantization profile": Q3G64_F16S, Q4G64_F16S, Q5G64_F16S
+// (group 64); [MXFP8] "Caveats": Q4/Q5/Q6 groupwise.
 // Per row r and group g: a = max |w| over the group (FP32); the stored scale
 // is s16 = binary16_rne(a / Qmax) with the FP32 quotient; s = value(s16);
 // q = (s == 0) ? 0 : clamp(rint(w / s), -(Qmax+1), Qmax), w / s in FP32.
-// Qmax = 7 (Q4), 15 (Q5), 127 (Q8, group 32).
+// Qmax = 2^(bits-1) - 1: 3 (Q3), 7 (Q4), 15 (Q5), 31 (Q6), 127 (Q8, group 32)
+// -- the signed range of the code width, as the pages' Q4/Q5 scale amax/7,
+// amax/15 read.
 // Pinned by: codes in range, |q*s - w| <= s/2, pack(dequant(pack)) == pack,
-// and the exhaustive codec tests.
+// hand-derived groups (ties included), and the exhaustive codec tests.
 int oracle_pack_groupwise(int fmt, const float* w, int64_t n, int64_t k, void* codes, void* hibits,
                           uint16_t* scales) {
-  if (fmt != FMT_Q4_G64 && fmt != FMT_Q5_G64 && fmt != FMT_Q8_G32) return 1;
+  if (!is_groupwise64(fmt) && fmt != FMT_Q8_G32) return 1;
   int gs = group_size(fmt);
   if (k % gs != 0 || (fmt != FMT_Q8_G32 && k % 64 != 0)) return 1;
-  int qmax = fmt == FMT_Q4_G64 ? 7 : (fmt == FMT_Q5_G64 ? 15 : 127);
+  int qmax = fmt == FMT_Q8_G32 ? 127 : code_offset(fmt) - 1;
   int64_t ng = k / gs;
-  if (fmt != FMT_Q8_G32) std::memset(codes, 0, (size_t)(n * (k / 2)));
-  if (fmt == FMT_Q5_G64) std::memset(hibits, 0, (size_t)(n * (k / 8)));
+  if (fmt == FMT_Q4_G64 || fmt == FMT_Q5_G64 || fmt == FMT_Q6_G64) std::memset(codes, 0, (size_t)(n * (k / 2)));
+  if (fmt == FMT_Q3_G64) std::memset(codes, 0, (size_t)(n * (k / 4)));
+  if (fmt == FMT_Q5_G64 || fmt == FMT_Q3_G64) std::memset(hibits, 0, (size_t)(n * (k / 8)));
+  if (fmt == FMT_Q6_G64) std::memset(hibits, 0, (size_t)(n * (k / 4)));
   for (int64_t r = 0; r < n; ++r) {
     for (int64_t g = 0; g < ng; ++g) {
       const float* wg = w + r * k + g * gs;
@@ -276,13 +316,20 @@ int oracle_pack_groupwise(int fmt, const float* w, int64_t n, int64_t k, void* c
         if (fmt == FMT_Q8_G32) {
           ((int8_t*)codes)[r * k + e] = (int8_t)q;
         } else {
-          int u = q + (fmt == FMT_Q4_G64 ? 8 : 16);
-          uint8_t* row = (uint8_t*)codes + r * (k / 2);
-          uint8_t* wp = row + (e / 8) * 4;
-          store_u32_le(wp, load_u32_le(wp) | ((uint32_t)(u & 0xF) << nibble_bit(e)));
-          if (fmt == FMT_Q5_G64) {
-            uint8_t* hp = (uint8_t*)hibits + r * (k / 8) + (e / 32) * 4;
-            store_u32_le(hp, load_u32_le(hp) | ((uint32_t)((u >> 4) & 1) << hibit_bit(e)));
+          const uint32_t u = (uint32_t)(q + code_offset(fmt));
+          // OR a field into a plane word (planes start zeroed)
+          auto put = [](uint8_t* wp, uint32_t field, int bit) {
+            store_u32_le(wp, load_u32_le(wp) | (field << bit));
+          };
+          uint8_t* cp = (uint8_t*)codes;
+          uint8_t* hp = (uint8_t*)hibits;
+          if (fmt == FMT_Q3_G64) {
+            put(cp + r * (k / 4) + (e / 16) * 4, u & 0x3, crumb_bit(e));
+            put(hp + r * (k / 8) + (e / 32) * 4, (u >> 2) & 1, hibit_bit(e));
+          } else {
+            put(cp + r * (k / 2) + (e / 8) * 4, u & 0xF, nibble_bit(e));
+            if (fmt == FMT_Q5_G64) put(hp + r * (k / 8) + (e / 32) * 4, (u >> 4) & 1, hibit_bit(e));
+            if (fmt == FMT_Q6_G64) put(hp + r * (k / 4) + (e / 16) * 4, (u >> 4) & 0x3, crumb_bit(e));
           }
         }
       }
@@ -471,7 +518,7 @@ int oracle_quantize_act(const uint16_t* x, int64_t t, int64_t k, int8_t* qa, flo
 // Pinned by: numpy integer matmul per group on tiny shapes; |S| at all-max codes.
 int oracle_group_sums(int fmt, const void* codes, const void* hibits, const int8_t* qa, int64_t t,
                       int64_t n, int64_t k, int32_t* S) {
-  if (fmt != FMT_Q4_G64 && fmt != FMT_Q5_G64) return 1;
+  if (!is_groupwise64(fmt)) return 1;
   int64_t ng = k / 64;
   for (int64_t tt = 0; tt < t; ++tt)
     for (int64_t r = 0; r < n; ++r)
@@ -496,7 +543,7 @@ int oracle_group_sums(int fmt, const void* codes, const void* hibits, const int8
 int oracle_gemm_a8(int fmt, const void* codes, const void* hibits, const uint16_t* wscales,
                    const int8_t* qa, const float* as, int64_t t, int64_t n, int64_t k, double* y,
                    double* bound, int nthreads) {
-  if (fmt != FMT_Q4_G64 && fmt != FMT_Q5_G64) return 1;
+  if (!is_groupwise64(fmt)) return 1;
   int64_t ng = k / 64;
   parallel_rows(n, nthreads, [&](int64_t r0, int64_t r1) {
     std::vector<int> qr((size_t)k);

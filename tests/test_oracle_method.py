@@ -7,9 +7,9 @@ import torch
 
 import synth
 
-Q4, Q5, Q8, FP8, BF16 = 0, 1, 2, 3, 4
-QMAX = {Q4: 7, Q5: 15, Q8: 127}
-GS = {Q4: 64, Q5: 64, Q8: 32}
+Q4, Q5, Q8, FP8, BF16, Q3, Q6 = 0, 1, 2, 3, 4, 5, 6
+QMAX = {Q4: 7, Q5: 15, Q8: 127, Q3: 3, Q6: 31}
+GS = {Q4: 64, Q5: 64, Q8: 32, Q3: 64, Q6: 64}
 
 
 def _bf16(x):
@@ -69,7 +69,8 @@ def _tie_row(ex, width):
     return v
 
 
-@pytest.mark.parametrize("name,fmt", [("q4_group", Q4), ("q5_group", Q5), ("q8_group", Q8)])
+@pytest.mark.parametrize("name,fmt", [("q4_group", Q4), ("q5_group", Q5), ("q8_group", Q8),
+                                      ("q3_group", Q3), ("q6_group", Q6)])
 def test_golden_pack_ties_round_half_even(orc, golden, name, fmt):
     """w/s exactly on k + 1/2: the codes are the even neighbours (a
     round-half-away-from-zero oracle fails here)."""
@@ -104,17 +105,40 @@ def test_page_constants_used(orc, golden):
 
 
 # ---- layouts: the documented bit positions ----------------------------------
+def _word(plane, r, i):
+    return int.from_bytes(plane[r, 4 * i:4 * i + 4].tobytes(), "little")
+
+
 def _layout_code(fmt, codes, hib, r, e):
     """Read element e of row r straight from the documented layout."""
-    w = int.from_bytes(codes[r, (e // 8) * 4:(e // 8) * 4 + 4].tobytes(), "little")
-    i = e % 8
-    u = (w >> (16 * (i % 2) + 4 * (i // 2))) & 0xF
+    if fmt == Q3:
+        i = e % 16
+        u = (_word(codes, r, e // 16) >> (16 * (i % 2) + 2 * (i // 2))) & 0x3
+    else:
+        i = e % 8
+        u = (_word(codes, r, e // 8) >> (16 * (i % 2) + 4 * (i // 2))) & 0xF
+    ee = e % 32
+    hbit = 16 * (ee % 2) + 4 * (ee // 8) + (ee % 8) // 2
     if fmt == Q5:
-        h = int.from_bytes(hib[r, (e // 32) * 4:(e // 32) * 4 + 4].tobytes(), "little")
-        ee = e % 32
-        u |= ((h >> (16 * (ee % 2) + 4 * (ee // 8) + (ee % 8) // 2)) & 1) << 4
-        return u - 16
+        return (u | (((_word(hib, r, e // 32) >> hbit) & 1) << 4)) - 16
+    if fmt == Q3:
+        return (u | (((_word(hib, r, e // 32) >> hbit) & 1) << 2)) - 4
+    if fmt == Q6:
+        i = e % 16
+        return (u | (((_word(hib, r, e // 16) >> (16 * (i % 2) + 2 * (i // 2))) & 0x3) << 4)) - 32
     return u - 8
+
+
+@pytest.mark.parametrize("name,fmt", [("q3_group", Q3), ("q6_group", Q6)])
+def test_golden_packed_words(orc, golden, name, fmt):
+    """The packed planes of the hand-derived tie groups, word for word."""
+    pw = orc.pack(fmt, _tie_row(golden["ties"][name], 64))
+    lay = golden["layouts"][name]
+    for key in ("codes", "hibits"):
+        plane = pw[key]
+        want = [int(h, 16) for h in lay[key + "_words"]]
+        assert plane.shape[1] == 4 * len(want), key
+        assert [_word(plane, 0, i) for i in range(len(want))] == want, key
 
 
 def _exact_codes_matrix(fmt, n, k, rng, scale_pow2=True):
@@ -129,7 +153,7 @@ def _exact_codes_matrix(fmt, n, k, rng, scale_pow2=True):
     return q, s, w
 
 
-@pytest.mark.parametrize("fmt", [Q4, Q5, Q8])
+@pytest.mark.parametrize("fmt", [Q4, Q5, Q8, Q3, Q6])
 def test_pack_exact_codes_and_layout(orc, fmt):
     rng = np.random.default_rng(10 + fmt)
     n, k = 5, 192
@@ -145,7 +169,7 @@ def test_pack_exact_codes_and_layout(orc, fmt):
     assert np.array_equal(orc.dequant(pw), w.astype(np.float64))
 
 
-@pytest.mark.parametrize("fmt", [Q4, Q5, Q8])
+@pytest.mark.parametrize("fmt", [Q4, Q5, Q8, Q3, Q6])
 def test_pack_half_step_bound_and_idempotence(orc, fmt):
     w = synth.weights_f32(24, 512, seed=77 + fmt).numpy()
     pw = orc.pack(fmt, w)
@@ -171,7 +195,7 @@ def test_pack_half_step_bound_and_idempotence(orc, fmt):
 def test_pack_zero_group(orc):
     w = np.zeros((2, 128), np.float32)
     w[1, 64:] = 0.25
-    for fmt in (Q4, Q5, Q8):
+    for fmt in (Q4, Q5, Q8, Q3, Q6):
         pw = orc.pack(fmt, w)
         assert np.all(orc.dequant(pw)[0] == 0)
         assert pw["scales"][0, 0] == 0
@@ -230,7 +254,7 @@ def test_mxfp8_synthetic_matches_closed_form(orc):
 
 
 # ---- GEMV ---------------------------------------------------------------------
-@pytest.mark.parametrize("fmt", [Q4, Q5, Q8])
+@pytest.mark.parametrize("fmt", [Q4, Q5, Q8, Q3, Q6])
 def test_gemv_unit_scales_is_integer_matmul(orc, fmt):
     rng = np.random.default_rng(20 + fmt)
     n, k, t = 7, 256, 3
@@ -297,7 +321,7 @@ def test_quantize_act_invariants(orc):
     assert np.all(top[as_ > 0] == 127)
 
 
-@pytest.mark.parametrize("fmt", [Q4, Q5])
+@pytest.mark.parametrize("fmt", [Q4, Q5, Q3, Q6])
 def test_group_sums_bruteforce(orc, fmt):
     rng = np.random.default_rng(30 + fmt)
     for k in (64, 128, 192):
@@ -311,7 +335,7 @@ def test_group_sums_bruteforce(orc, fmt):
             assert np.array_equal(S[:, :, g], ref)
 
 
-@pytest.mark.parametrize("fmt", [Q4, Q5])
+@pytest.mark.parametrize("fmt", [Q4, Q5, Q3, Q6])
 def test_group_sums_extremes(orc, fmt):
     qmax = QMAX[fmt]
     for sign_w, sign_a in ((1, 1), (-1, 1), (1, -1)):
@@ -322,7 +346,7 @@ def test_group_sums_extremes(orc, fmt):
         assert np.all(S == sign_w * sign_a * 64 * qmax * 127)
 
 
-@pytest.mark.parametrize("fmt", [Q4, Q5])
+@pytest.mark.parametrize("fmt", [Q4, Q5, Q3, Q6])
 def test_gemm_a8_unit_scales_is_integer_matmul(orc, fmt):
     rng = np.random.default_rng(40 + fmt)
     n, k, t = 6, 192, 4
@@ -341,7 +365,7 @@ def test_gemm_a8_scaled_matches_group_sums(orc):
     """With real scales: y = sum_g FP32(ws*as) * S_g (numpy FP32 product)."""
     w = synth.weights_f32(12, 320, seed=50).numpy()
     x = synth.activations_bf16(6, 320, seed=51).view(torch.int16).numpy().view(np.uint16)
-    for fmt in (Q4, Q5):
+    for fmt in (Q4, Q5, Q3, Q6):
         pw = orc.pack(fmt, w)
         qa, as_ = orc.quantize_act(x)
         S = orc.group_sums(pw, qa).astype(np.float64)
