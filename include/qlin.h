@@ -32,7 +32,7 @@
  *     legacy default stream).  Argument checks happen on the host before
  *     anything is enqueued; a rejected call enqueues nothing.
  *   - Every device array must start on a 16-byte boundary (TMA rule), and
- *     K must be a multiple of the format's group (64 for Q4/Q5, 32 for Q8,
+ *     K must be a multiple of the format's group (64 for Q3/Q4/Q5/Q6, 32 for Q8,
  *     32 for MXFP8 sources, 128 for MLX affine sources, 64 for BF16/FP8 rows).
  *   - Kernels that wait on on-chip barriers bound every wait.  A wait that
  *     runs out stores QLIN_ERR_TIMEOUT into `*qlin_exec.dev_status` (when the
@@ -54,6 +54,19 @@
  *           scales binary16[N][K/32].
  *   FP8_ROW codes E4M3 bytes [N][K]; scales bfloat16[N] (one per row).
  *   BF16    codes bfloat16[N][K]; no scales.
+ *   Q3_G64  u = q + 4, q in [-4, 3] (scale amax / 3).  codes uint8[N][K/4],
+ *           the crumb plane of bits 0..1 of u: read as K/16 little-endian
+ *           words, word c holds element 16c + 2s + o (s in 0..7, o in 0..1)
+ *           in bits [16o + 2s, 16o + 2s + 2); hibits uint8[N][K/8], bit 2 of
+ *           u laid out as Q5's high-bit plane.  scales binary16[N][K/64].
+ *   Q6_G64  u = q + 32, q in [-32, 31] (scale amax / 31).  codes as Q4
+ *           holding bits 0..3 of u; hibits uint8[N][K/4], bits 4..5 of u in
+ *           the crumb layout of Q3's codes.  scales binary16[N][K/64].
+ *           ["Qwen3.8-27B for NInfer -- RTX 5080 16 GB", "Quantization
+ *           profile": Q3G64_F16S; "Qwen3.8-27B MXFP8-CRACK -- NInfer
+ *           artifact", "Caveats": Q6 groupwise.  The code widths and group
+ *           size are the pages'; Qmax = 2^(bits-1) - 1 and the planes are this
+ *           library's reading.]
  * Activations x are bfloat16[T][K] row-major; outputs y are [T][N] row-major
  * in bfloat16 or float32 (y[t][n] = sum_k w[n][k] * x[t][k]).
  */
@@ -88,6 +101,8 @@ extern "C" {
 #define QLIN_Q8_G32 2
 #define QLIN_FP8_ROW 3
 #define QLIN_BF16 4
+#define QLIN_Q3_G64 5
+#define QLIN_Q6_G64 6
 
 /* ---- weight sources for qlin_pack_weights ------------------------------- */
 #define QLIN_SRC_F32 0         /* float32[N][K]                                 */
@@ -196,7 +211,7 @@ QLIN_API int qlin_gemv(const qlin_weights* w, const uint16_t* x_bf16, int64_t t,
 /* Workspace bytes qlin_gemm_a8 needs for T tokens against an N x K matrix. */
 QLIN_API int qlin_gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, size_t* bytes);
 
-/* Int8-route projection (prefill).  Weights must be Q4_G64 or Q5_G64
+/* Int8-route projection (prefill).  Weights must be Q3_G64, Q4_G64, Q5_G64 or Q6_G64
  * (QLIN_ERR_UNSUPPORTED otherwise) carrying QLIN_ALLOW_A8
  * (QLIN_ERR_NOT_PERMITTED otherwise) and K % 128 == 0 (QLIN_ERR_UNSUPPORTED
  * otherwise).  Activations either as x_bf16 (the

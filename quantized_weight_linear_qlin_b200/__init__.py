@@ -12,7 +12,7 @@ import os
 import torch
 
 __all__ = [
-    "QlinError", "Q4_G64", "Q5_G64", "Q8_G32", "FP8_ROW", "BF16",
+    "QlinError", "Q4_G64", "Q5_G64", "Q8_G32", "FP8_ROW", "BF16", "Q3_G64", "Q6_G64",
     "SRC_F32", "SRC_BF16", "SRC_MXFP8", "SRC_MLX_AFFINE8", "SRC_FP8_BLOCK128", "OUT_BF16", "OUT_F32",
     "ALLOW_A8", "DEBUG_GROUP_SUMS", "PackedWeights", "Workspace", "lib",
     "qlin_packed_bytes", "qlin_pack_weights", "qlin_decode_mxfp8", "qlin_quantize_act",
@@ -21,7 +21,7 @@ __all__ = [
     "qlin_gemm_fp8_workspace_bytes", "qlin_gemm_fp8",
 ]
 
-Q4_G64, Q5_G64, Q8_G32, FP8_ROW, BF16 = 0, 1, 2, 3, 4
+Q4_G64, Q5_G64, Q8_G32, FP8_ROW, BF16, Q3_G64, Q6_G64 = 0, 1, 2, 3, 4, 5, 6
 SRC_F32, SRC_BF16, SRC_MXFP8, SRC_MLX_AFFINE8, SRC_FP8_BLOCK128 = 0, 1, 2, 3, 4
 OUT_BF16, OUT_F32 = 0, 1
 ALLOW_A8 = 0x1

@@ -80,8 +80,10 @@ thread_local TmapCache t_tmaps;
 
 int group_of(int fmt) {
   switch (fmt) {
+    case QLIN_Q3_G64:
     case QLIN_Q4_G64:
     case QLIN_Q5_G64:
+    case QLIN_Q6_G64:
     case QLIN_FP8_ROW:
     case QLIN_BF16:
       return 64;
@@ -99,6 +101,8 @@ int sizes_of(int fmt, int64_t n, int64_t k, size_t* c, size_t* h, size_t* s) {
   switch (fmt) {
     case QLIN_Q4_G64: cb = (size_t)n * (k / 2); sb = (size_t)n * (k / 64) * 2; break;
     case QLIN_Q5_G64: cb = (size_t)n * (k / 2); hb = (size_t)n * (k / 8); sb = (size_t)n * (k / 64) * 2; break;
+    case QLIN_Q3_G64: cb = (size_t)n * (k / 4); hb = (size_t)n * (k / 8); sb = (size_t)n * (k / 64) * 2; break;
+    case QLIN_Q6_G64: cb = (size_t)n * (k / 2); hb = (size_t)n * (k / 4); sb = (size_t)n * (k / 64) * 2; break;
     case QLIN_Q8_G32: cb = (size_t)n * k; sb = (size_t)n * (k / 32) * 2; break;
     case QLIN_FP8_ROW: cb = (size_t)n * k; sb = (size_t)n * 2; break;
     case QLIN_BF16: cb = (size_t)n * k * 2; break;
@@ -318,7 +322,8 @@ int qlin_gemm_a8(const qlin_weights* w, const uint16_t* x_bf16, const int8_t* xq
                  const qlin_exec* ex) {
   int rc = check_weights(w);
   if (rc) return rc;
-  if (w->fmt != QLIN_Q4_G64 && w->fmt != QLIN_Q5_G64) return QLIN_ERR_UNSUPPORTED;
+  if (w->fmt != QLIN_Q4_G64 && w->fmt != QLIN_Q5_G64 && w->fmt != QLIN_Q3_G64 && w->fmt != QLIN_Q6_G64)
+    return QLIN_ERR_UNSUPPORTED;
   if (!(w->flags & QLIN_ALLOW_A8)) return QLIN_ERR_NOT_PERMITTED;
   if (w->k % 128) return QLIN_ERR_UNSUPPORTED;
   if (t <= 0 || !y || !aligned16(y)) return QLIN_ERR_INVALID_ARG;

@@ -87,7 +87,6 @@ constexpr int BM = 128;         // weight rows per tile (tensor-memory lanes)
 constexpr int BN = 128;         // tokens per tile (accumulator columns)
 constexpr int BKC = 256;        // K columns per pipeline stage (four 64-groups)
 constexpr int GPS = BKC / 64;   // groups per stage
-constexpr int STAGES = 4;
 constexpr int NDS = 2;          // group-sum slots (128 columns each)
 constexpr int NAS = 8;          // A slots (one group of int8 codes: 16 columns each)
 constexpr int Y_COL0 = NDS * BN;        // the tile's FP32 output accumulator (128 columns)
@@ -103,16 +102,30 @@ constexpr int NUM_THREADS = 16 * 32;
 constexpr uint32_t ACC_BIAS = 0x4B400000u;
 constexpr float ACC_BIAS_F = 12582912.0f;
 
+// Per code width: bytes per row and stage (256 columns) of the code plane and
+// of the second plane, and the pipeline depth that fits shared memory.
+//   Q3: crumb plane 64 B (unswizzled) + bit plane 32 B;  Q4: nibble plane
+//   128 B (128-byte swizzle);  Q5: + bit plane 32 B;  Q6: + crumb plane 64 B.
+template <int BITS>
+struct A8Fmt {
+  static constexpr int RAW_ROW = BITS == 3 ? 64 : 128;
+  static constexpr int HIB_ROW = BITS == 6 ? 64 : (BITS == 3 || BITS == 5) ? 32 : 0;
+  static constexpr int STAGES = BITS == 6 ? 3 : 4;
+};
+
+template <int BITS>
 struct __align__(1024) StageSmem {
   uint8_t b[2][BN * 128];        // int8 activations, two 128-column swizzled atoms
-  uint8_t raw[BM * 128];         // packed nibbles of 256 columns (swizzled)
-  uint8_t hib[BM * 32];          // Q5 high bits of 256 columns
+  uint8_t raw[BM * 128];         // code plane of 256 columns
+  uint8_t hib[BM * (A8Fmt<BITS>::HIB_ROW ? A8Fmt<BITS>::HIB_ROW : 16)];  // second plane
   float xsb[GPS * BN];           // activation scales of the stage, [group][token]
   __half wsb[BM * GPS];          // weight scales of the stage, [row][group]
 };
 
+template <int BITS>
 struct Smem {
-  StageSmem st[STAGES];
+  static constexpr int STAGES = A8Fmt<BITS>::STAGES;
+  StageSmem<BITS> st[STAGES];
   uint64_t full[STAGES], empty[STAGES];
   uint64_t a_full[NAS], a_free[NAS];
   uint64_t d_full[NDS], d_empty[NDS];
@@ -132,11 +145,13 @@ struct GemmArgs {
   int y_dtype;
 };
 
-__device__ __forceinline__ void set_abort(Smem& sm, int32_t* dev_status) {
+template <class SM>
+__device__ __forceinline__ void set_abort(SM& sm, int32_t* dev_status) {
   *(volatile int*)&sm.abort_flag = 1;
   report_timeout(dev_status);
 }
-__device__ __forceinline__ bool aborted(Smem& sm) { return *(volatile int*)&sm.abort_flag != 0; }
+template <class SM>
+__device__ __forceinline__ bool aborted(SM& sm) { return *(volatile int*)&sm.abort_flag != 0; }
 
 // A ring position: slot index and the parity of its current use.
 struct Ring {
@@ -149,27 +164,88 @@ struct Ring {
   }
 };
 
-// Expand 8 nibbles of one layout word into 8 signed int8 codes in element order.
+// Expand 8 nibbles of one layout word into the offset codes u (bytes, element
+// order): element 8j+2s+o sits at bits 16o+4s.  `b0`, `b1` are the higher bits
+// of u already in place (bit 4 and up of each byte).
+__device__ __forceinline__ uint2 nibble_bytes(uint32_t w) {
+  const uint32_t lo = w & 0x0F0F0F0Fu;         // elements 0, 4, 1, 5
+  const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // elements 2, 6, 3, 7
+  return make_uint2(__byte_perm(lo, hi, 0x6420),   // elements 0..3
+                    __byte_perm(lo, hi, 0x7531));  // elements 4..7
+}
+
+// One 64-group of row r as 64 signed int8 codes q = u - 2^(BITS-1) in element
+// order (16 words).  `raw` is the stage's code plane (128-byte swizzled
+// nibbles, or for Q3 unswizzled 64-byte crumb rows), `hib` its second plane.
 template <int BITS>
-__device__ __forceinline__ uint2 expand_word(uint32_t w, uint32_t h) {
-  uint32_t lo = w & 0x0F0F0F0Fu;         // elements 0, 4, 1, 5
-  uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // elements 2, 6, 3, 7
-  uint32_t o0 = __byte_perm(lo, hi, 0x6420);  // elements 0..3
-  uint32_t o1 = __byte_perm(lo, hi, 0x7531);  // elements 4..7
-  if constexpr (BITS == 4) {
-    o0 = (o0 + 0x78787878u) ^ 0x80808080u;
-    o1 = (o1 + 0x78787878u) ^ 0x80808080u;
+__device__ __forceinline__ void expand_group(const uint8_t* raw, const uint8_t* hib, int r, int gi,
+                                             uint32_t* o) {
+  // u + (128 - 2^(BITS-1)) then flip bit 7: the two's complement byte of q
+  constexpr uint32_t ADD = BITS == 3 ? 0x7C7C7C7Cu : BITS == 4 ? 0x78787878u : BITS == 5 ? 0x70707070u
+                                                                             : 0x60606060u;
+  if constexpr (BITS == 3) {
+    const uint4 c = *(const uint4*)(raw + r * 64 + gi * 16);  // 4 crumb words: elements 16cw + 2s + o
+    const uint2 hh = *(const uint2*)(hib + r * 32 + gi * 8);  // bit words: elements 0..31, 32..63
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int cw = 0; cw < 4; ++cw) {
+      const uint32_t m0 = w[cw] & 0x03030303u;         // elements 0, 8, 1, 9
+      const uint32_t m1 = (w[cw] >> 2) & 0x03030303u;  // 2, 10, 3, 11
+      const uint32_t m2 = (w[cw] >> 4) & 0x03030303u;  // 4, 12, 5, 13
+      const uint32_t m3 = (w[cw] >> 6) & 0x03030303u;  // 6, 14, 7, 15
+      const uint32_t e[4] = {__byte_perm(m0, m1, 0x6420), __byte_perm(m2, m3, 0x6420),
+                             __byte_perm(m0, m1, 0x7531), __byte_perm(m2, m3, 0x7531)};
+      // bit of element 2s+o of this crumb word: bit 16o + s of Hc
+      const uint32_t Hc = (cw < 2 ? hh.x : hh.y) >> (8 * (cw & 1));
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t Hq = Hc >> (2 * q);  // elements 4q, 4q+1, 4q+2, 4q+3 at bits 0, 16, 1, 17
+        const uint32_t b = ((Hq << 2) & 0x4u) | ((Hq >> 6) & 0x400u) | ((Hq << 17) & 0x40000u) |
+                           ((Hq << 9) & 0x4000000u);
+        o[4 * cw + q] = ((e[q] | b) + ADD) ^ 0x80808080u;
+      }
+    }
   } else {
-    // h: this word's high bits shifted down to bits {0..3} (o = 0) and {16..19} (o = 1);
-    // element 2s+o needs its bit at byte (2s+o) % 4, bit 4.
-    uint32_t b0 = ((h << 4) & 0x10u) | ((h >> 4) & 0x1000u) | ((h << 19) & 0x100000u) |
-                  ((h << 11) & 0x10000000u);
-    uint32_t b1 = ((h << 2) & 0x10u) | ((h >> 6) & 0x1000u) | ((h << 17) & 0x100000u) |
-                  ((h << 9) & 0x10000000u);
-    o0 = ((o0 | b0) + 0x70707070u) ^ 0x80808080u;
-    o1 = ((o1 | b1) + 0x70707070u) ^ 0x80808080u;
+    uint32_t h[4] = {0u, 0u, 0u, 0u};
+    if constexpr (BITS == 5) {
+      const uint2 hh = *(const uint2*)(hib + r * 32 + gi * 8);
+      h[0] = hh.x;
+      h[1] = hh.y;
+    } else if constexpr (BITS == 6) {
+      const uint4 hh = *(const uint4*)(hib + r * 64 + gi * 16);  // crumb words of elements 16c..
+      h[0] = hh.x;
+      h[1] = hh.y;
+      h[2] = hh.z;
+      h[3] = hh.w;
+    }
+#pragma unroll
+    for (int uu = 0; uu < 2; ++uu) {  // 16-byte units 2gi, 2gi+1 of the row = 64 elements
+      const uint4 c = *(const uint4*)(raw + sw128_offset(r, 2 * gi + uu));
+      const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int jw = 4 * uu + j;  // nibble word of the group: elements 8jw..8jw+7
+        uint2 e = nibble_bytes(wv[j]);
+        if constexpr (BITS == 5) {
+          // bit of element 8jw+2s+o at 16o + 4(jw&3) + s of word jw/4 -> bit 4 of its byte
+          const uint32_t hw = h[uu] >> (4 * j);
+          e.x |= ((hw << 4) & 0x10u) | ((hw >> 4) & 0x1000u) | ((hw << 19) & 0x100000u) |
+                 ((hw << 11) & 0x10000000u);
+          e.y |= ((hw << 2) & 0x10u) | ((hw >> 6) & 0x1000u) | ((hw << 17) & 0x100000u) |
+                 ((hw << 9) & 0x10000000u);
+        } else if constexpr (BITS == 6) {
+          // crumb of element 8jw+2s+o at 16o + 8(jw&1) + 2s of word jw/2 -> bits 4..5 of its byte
+          const uint32_t cj = h[jw >> 1] >> (8 * (jw & 1));
+          e.x |= ((cj << 4) & 0x30u) | ((cj >> 4) & 0x3000u) | ((cj << 18) & 0x300000u) |
+                 ((cj << 10) & 0x30000000u);
+          e.y |= (cj & 0x30u) | ((cj >> 8) & 0x3000u) | ((cj << 14) & 0x300000u) |
+                 ((cj << 6) & 0x30000000u);
+        }
+        o[8 * uu + 2 * j] = (e.x + ADD) ^ 0x80808080u;
+        o[8 * uu + 2 * j + 1] = (e.y + ADD) ^ 0x80808080u;
+      }
+    }
   }
-  return make_uint2(o0, o1);
 }
 
 template <int BITS, bool DEBUG>
@@ -177,8 +253,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_a8_kernel(const __grid_constant__ CUtensorMap tm_codes,
                    const __grid_constant__ CUtensorMap tm_hib,
                    const __grid_constant__ CUtensorMap tm_act, GemmArgs args) {
+  using F = A8Fmt<BITS>;
+  constexpr int STAGES = F::STAGES;
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((void*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023));
+  Smem<BITS>& sm = *reinterpret_cast<Smem<BITS>*>((void*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ng = args.k / 64;
   const int nchunks = (int)((args.k + BKC - 1) / BKC);
@@ -210,7 +288,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == WARP_TMA && lane == 0) {
     tma_prefetch_desc(&tm_codes);
     tma_prefetch_desc(&tm_act);
-    if (BITS == 5) tma_prefetch_desc(&tm_hib);
+    if (F::HIB_ROW) tma_prefetch_desc(&tm_hib);
   }
   tc_fence_before();
   __syncthreads();
@@ -248,10 +326,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const int gcount = (int)min((int64_t)GPS, ng - (int64_t)kc * GPS);
         if (lane == 0) {
-          uint32_t bytes = BM * 128 + 2 * BN * 128 + (BITS == 5 ? BM * 32 : 0);
+          uint32_t bytes = BM * F::RAW_ROW + 2 * BN * 128 + BM * F::HIB_ROW;
           mbar_arrive_expect_tx(&sm.full[s], bytes);
-          tma_load_2d(sm.st[s].raw, &tm_codes, &sm.full[s], kc * 128, (int)n0);
-          if (BITS == 5) tma_load_2d(sm.st[s].hib, &tm_hib, &sm.full[s], kc * 32, (int)n0);
+          tma_load_2d(sm.st[s].raw, &tm_codes, &sm.full[s], kc * F::RAW_ROW, (int)n0);
+          if (F::HIB_ROW) tma_load_2d(sm.st[s].hib, &tm_hib, &sm.full[s], kc * F::HIB_ROW, (int)n0);
           tma_load_2d(sm.st[s].b[0], &tm_act, &sm.full[s], kc * BKC, (int)t0);
           tma_load_2d(sm.st[s].b[1], &tm_act, &sm.full[s], kc * BKC + 128, (int)t0);
         }
@@ -340,23 +418,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          uint2 hw = make_uint2(0, 0);  // Q5: the high-bit words of units 2gi, 2gi+1
-          if (BITS == 5) hw = *(const uint2*)(sm.st[s].hib + r * 32 + gi * 8);
           uint32_t o[16];
-#pragma unroll
-          for (int uu = 0; uu < 2; ++uu) {  // 16-byte units 2gi, 2gi+1 of the row = 64 elements
-            const int u = 2 * gi + uu;
-            const uint4 c = *(const uint4*)(raw + sw128_offset(r, u));
-            const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint32_t h = 0;
-              if (BITS == 5) h = (uu ? hw.y : hw.x) >> (4 * j);
-              const uint2 e = expand_word<BITS>(wv[j], h);
-              o[8 * uu + 2 * j] = e.x;
-              o[8 * uu + 2 * j + 1] = e.y;
-            }
-          }
+          expand_group<BITS>(raw, sm.st[s].hib, r, gi, o);
           tmem_st_x16(tmem + lane_ofs + A_COL0 + ar.slot * 16, o);
           tmem_st_wait();
           tc_fence_before();
@@ -522,6 +585,25 @@ int launch_quantize_act(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, flo
   return cuda_status(cudaGetLastError());
 }
 
+template <int BITS, bool DEBUG>
+static int launch_a8(const CUtensorMap& tm_codes, const CUtensorMap& tm_hib, const CUtensorMap& tm_act,
+                     const GemmArgs& args, int grid, const Exec& ex) {
+  const size_t smem = sizeof(Smem<BITS>) + 1024;
+  const cudaError_t e0 = set_smem_once<gemm_a8_kernel<BITS, DEBUG>>((int)smem);
+  if (e0 != cudaSuccess) return cuda_status(e0);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = ex.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, gemm_a8_kernel<BITS, DEBUG>, tm_codes, tm_hib, tm_act, args));
+}
+
 int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, const float* xs,
                    int64_t t, void* y, int y_dtype, uint32_t flags, int32_t* sums_dbg,
                    const Exec& ex) {
@@ -535,16 +617,22 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
     xq = wq;
     xs = wsc;
   }
+  const int bits = w.fmt == QLIN_Q3_G64 ? 3 : w.fmt == QLIN_Q4_G64 ? 4 : w.fmt == QLIN_Q5_G64 ? 5 : 6;
+  // code plane: 128-byte swizzled nibble rows, or (Q3) unswizzled 64-byte crumb rows per stage
+  const uint64_t crow = (uint64_t)(bits == 3 ? k / 4 : k / 2);
   CUtensorMap tm_codes, tm_hib, tm_act;
-  int rc = encode_tmap_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, (uint64_t)(k / 2),
-                          (uint64_t)n, (uint64_t)(k / 2), 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  int rc = encode_tmap_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, crow, (uint64_t)n, crow,
+                          bits == 3 ? 64 : 128, BM,
+                          bits == 3 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   rc = encode_tmap_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)k, (uint64_t)t,
                       (uint64_t)k, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
-  if (w.fmt == QLIN_Q5_G64) {
-    rc = encode_tmap_2d(&tm_hib, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.hibits, (uint64_t)(k / 8),
-                        (uint64_t)n, (uint64_t)(k / 8), 32, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (bits != 4) {
+    // second plane: 32 (bit plane) or 64 (crumb plane) bytes per row per stage
+    const uint64_t hrow = (uint64_t)(bits == 6 ? k / 4 : k / 8);
+    rc = encode_tmap_2d(&tm_hib, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.hibits, hrow, (uint64_t)n, hrow,
+                        bits == 6 ? 64 : 32, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
   } else {
     tm_hib = tm_codes;
@@ -562,29 +650,17 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
   args.tiles = args.tiles_t * ((n + BM - 1) / BM);
   args.y_dtype = y_dtype;
   const bool debug = (flags & QLIN_DEBUG_GROUP_SUMS) != 0;
-
-  const size_t smem = sizeof(Smem) + 1024;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)std::min<int64_t>(args.tiles, ex.num_sms));
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = ex.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e;
-  auto kern = w.fmt == QLIN_Q4_G64 ? (debug ? gemm_a8_kernel<4, true> : gemm_a8_kernel<4, false>)
-                                    : (debug ? gemm_a8_kernel<5, true> : gemm_a8_kernel<5, false>);
-  e = w.fmt == QLIN_Q4_G64
-          ? (debug ? set_smem_once<gemm_a8_kernel<4, true>>((int)smem)
-                   : set_smem_once<gemm_a8_kernel<4, false>>((int)smem))
-          : (debug ? set_smem_once<gemm_a8_kernel<5, true>>((int)smem)
-                   : set_smem_once<gemm_a8_kernel<5, false>>((int)smem));
-  if (e != cudaSuccess) return cuda_status(e);
-  e = cudaLaunchKernelEx(&cfg, kern, tm_codes, tm_hib, tm_act, args);
-  return cuda_status(e);
+  const int grid = (int)std::min<int64_t>(args.tiles, ex.num_sms);
+  switch (bits) {
+    case 3: return debug ? launch_a8<3, true>(tm_codes, tm_hib, tm_act, args, grid, ex)
+                         : launch_a8<3, false>(tm_codes, tm_hib, tm_act, args, grid, ex);
+    case 4: return debug ? launch_a8<4, true>(tm_codes, tm_hib, tm_act, args, grid, ex)
+                         : launch_a8<4, false>(tm_codes, tm_hib, tm_act, args, grid, ex);
+    case 5: return debug ? launch_a8<5, true>(tm_codes, tm_hib, tm_act, args, grid, ex)
+                         : launch_a8<5, false>(tm_codes, tm_hib, tm_act, args, grid, ex);
+    default: return debug ? launch_a8<6, true>(tm_codes, tm_hib, tm_act, args, grid, ex)
+                          : launch_a8<6, false>(tm_codes, tm_hib, tm_act, args, grid, ex);
+  }
 }
 
 }  // namespace qlin

@@ -30,6 +30,10 @@ struct Traits<QLIN_Q4_G64> { static constexpr int EPC = 32, GS = 64; };
 template <>
 struct Traits<QLIN_Q5_G64> { static constexpr int EPC = 32, GS = 64; };
 template <>
+struct Traits<QLIN_Q3_G64> { static constexpr int EPC = 64, GS = 64; };
+template <>
+struct Traits<QLIN_Q6_G64> { static constexpr int EPC = 32, GS = 64; };
+template <>
 struct Traits<QLIN_Q8_G32> { static constexpr int EPC = 16, GS = 32; };
 template <>
 struct Traits<QLIN_FP8_ROW> { static constexpr int EPC = 16, GS = 0; };
@@ -41,13 +45,14 @@ __device__ __forceinline__ float u_to_q(uint32_t u, float off_plus_magic) {
   return __uint_as_float(0x4B000000u | u) - off_plus_magic;
 }
 
-// Decode one 16-byte chunk into EPC exact weight values (codes, not yet scaled).
+// Decode one 16-byte chunk of the code plane (plus the matching second-plane
+// words hw) into EPC exact weight values (codes, not yet scaled).
 // Element order: out[e] is element e of the chunk.
 template <int FMT>
-__device__ __forceinline__ void decode_chunk(uint4 c, uint32_t hw, float* out) {
+__device__ __forceinline__ void decode_chunk(uint4 c, uint2 hw, float* out) {
   uint32_t w[4] = {c.x, c.y, c.z, c.w};
-  if constexpr (FMT == QLIN_Q4_G64 || FMT == QLIN_Q5_G64) {
-    constexpr float OFFM = FMT == QLIN_Q4_G64 ? 8388608.0f + 8.0f : 8388608.0f + 16.0f;
+  if constexpr (FMT == QLIN_Q4_G64 || FMT == QLIN_Q5_G64 || FMT == QLIN_Q6_G64) {
+    constexpr float OFFM = 8388608.0f + (FMT == QLIN_Q4_G64 ? 8.0f : FMT == QLIN_Q5_G64 ? 16.0f : 32.0f);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
 #pragma unroll
@@ -55,8 +60,27 @@ __device__ __forceinline__ void decode_chunk(uint4 c, uint32_t hw, float* out) {
 #pragma unroll
         for (int o = 0; o < 2; ++o) {
           uint32_t u = (w[j] >> (16 * o + 4 * s)) & 0xFu;
-          if constexpr (FMT == QLIN_Q5_G64) u |= ((hw >> (16 * o + 4 * j + s)) & 1u) << 4;
+          // Q5: bit of element 8j+2s+o at 16o+4j+s; Q6: crumb of element
+          // 8j+2s+o in word j/2 at bits 16o + 8(j&1) + 2s
+          if constexpr (FMT == QLIN_Q5_G64) u |= ((hw.x >> (16 * o + 4 * j + s)) & 1u) << 4;
+          if constexpr (FMT == QLIN_Q6_G64)
+            u |= (((j < 2 ? hw.x : hw.y) >> (16 * o + 8 * (j & 1) + 2 * s)) & 3u) << 4;
           out[8 * j + 2 * s + o] = u_to_q(u, OFFM);
+        }
+      }
+    }
+  } else if constexpr (FMT == QLIN_Q3_G64) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+#pragma unroll
+        for (int o = 0; o < 2; ++o) {
+          // crumb of element 16j+2s+o at 16o+2s; its bit in word j/2 at
+          // 16o + 8(j&1) + 4(s>>2) + (s&3)
+          uint32_t u = (w[j] >> (16 * o + 2 * s)) & 3u;
+          u |= (((j < 2 ? hw.x : hw.y) >> (16 * o + 8 * (j & 1) + 4 * (s >> 2) + (s & 3))) & 1u) << 2;
+          out[16 * j + 2 * s + o] = u_to_q(u, 8388608.0f + 4.0f);
         }
       }
     }
@@ -101,13 +125,15 @@ __global__ void __launch_bounds__(kThreads) gemv_cc_kernel(
     const void* __restrict__ scales, const uint16_t* __restrict__ x, int64_t n, int64_t k, int64_t t,
     int64_t krange, void* __restrict__ y, int y_dtype, float* __restrict__ acc_ws) {
   constexpr int EPC = Traits<FMT>::EPC;
-  constexpr int BPE = FMT == QLIN_BF16 ? 2 : (FMT == QLIN_Q8_G32 || FMT == QLIN_FP8_ROW ? 1 : 0);
+  // code-plane bits per element
+  constexpr int CB = FMT == QLIN_BF16 ? 16 : (FMT == QLIN_Q8_G32 || FMT == QLIN_FP8_ROW) ? 8
+                     : FMT == QLIN_Q3_G64 ? 2 : 4;
   extern __shared__ float xs[];  // [kTokBlock][krange]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t k0 = (int64_t)blockIdx.y * krange;
   const int64_t k1 = min(k, k0 + krange);
   const int64_t kr = k1 - k0;
-  const int64_t row_bytes = BPE == 0 ? k / 2 : k * BPE;
+  const int64_t row_bytes = k * CB / 8;
   const bool split = gridDim.y > 1;
 
   for (int64_t t0 = 0; t0 < t; t0 += kTokBlock) {
@@ -134,13 +160,11 @@ __global__ void __launch_bounds__(kThreads) gemv_cc_kernel(
         for (int rr = 0; rr < kRowsPerWarp; ++rr) {
           const int64_t r = r0 + rr;
           if (r >= n) break;
-          uint4 c;
-          if constexpr (BPE == 0)
-            c = __ldcs((const uint4*)(codes + r * row_bytes + e0 / 2));
-          else
-            c = __ldcs((const uint4*)(codes + r * row_bytes + e0 * BPE));
-          uint32_t hw = 0;
-          if constexpr (FMT == QLIN_Q5_G64) hw = __ldcs((const uint32_t*)(hibits + r * (k / 8) + e0 / 8));
+          const uint4 c = __ldcs((const uint4*)(codes + r * row_bytes + e0 * CB / 8));
+          uint2 hw = make_uint2(0u, 0u);
+          if constexpr (FMT == QLIN_Q5_G64) hw.x = __ldcs((const uint32_t*)(hibits + r * (k / 8) + e0 / 8));
+          if constexpr (FMT == QLIN_Q3_G64) hw = __ldcs((const uint2*)(hibits + r * (k / 8) + e0 / 8));
+          if constexpr (FMT == QLIN_Q6_G64) hw = __ldcs((const uint2*)(hibits + r * (k / 4) + e0 / 4));
           float wv[EPC];
           decode_chunk<FMT>(c, hw, wv);
           const float sc = group_scale<FMT>(scales, r, k, e0);
@@ -244,6 +268,8 @@ int launch_gemv_cc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
   switch (w.fmt) {
     case QLIN_Q4_G64: return launch_cc<QLIN_Q4_G64>(w, x, t, y, y_dtype, ex, acc_ws);
     case QLIN_Q5_G64: return launch_cc<QLIN_Q5_G64>(w, x, t, y, y_dtype, ex, acc_ws);
+    case QLIN_Q3_G64: return launch_cc<QLIN_Q3_G64>(w, x, t, y, y_dtype, ex, acc_ws);
+    case QLIN_Q6_G64: return launch_cc<QLIN_Q6_G64>(w, x, t, y, y_dtype, ex, acc_ws);
     case QLIN_Q8_G32: return launch_cc<QLIN_Q8_G32>(w, x, t, y, y_dtype, ex, acc_ws);
     case QLIN_FP8_ROW: return launch_cc<QLIN_FP8_ROW>(w, x, t, y, y_dtype, ex, acc_ws);
     case QLIN_BF16: return launch_cc<QLIN_BF16>(w, x, t, y, y_dtype, ex, acc_ws);

@@ -40,7 +40,7 @@ struct SmCfg {
   static constexpr int KC = Tr::GK * GPC;             // K columns per unit
   static constexpr int XBOXES = KC / 64;              // activation boxes (64 columns x T rows)
   static constexpr int X_BYTES = XBOXES * T * 128;
-  static constexpr int HIB_BYTES = Tr::HIB ? UBS * 128 * 32 : 0;
+  static constexpr int HIB_BYTES = Tr::HIB ? UBS * 128 * Tr::HROW : 0;
   static constexpr int SC_ROW = Tr::PER_GROUP ? GPC * 2 : 0;
   static constexpr int SC_BYTES = 128 * SC_ROW;
   static constexpr int TMA_BYTES = UBS * BOX_BYTES + X_BYTES + HIB_BYTES;
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
 #pragma unroll
         for (int b = 0; b < UBS; ++b)
           tma_load_2d(st + b * BOX_BYTES, &tm_codes, &full[s], (ch * UBS + b) * 128, tile * 128);
-        if (Tr::HIB) tma_load_2d(st + C::OFF_HIB, &tm_hib, &full[s], ch * UBS * 32, tile * 128);
+        if (Tr::HIB) tma_load_2d(st + C::OFF_HIB, &tm_hib, &full[s], ch * UBS * Tr::HROW, tile * 128);
 #pragma unroll
         for (int b = 0; b < C::XBOXES; ++b)
           tma_load_2d(st + C::OFF_X + b * T * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0);
@@ -157,8 +157,9 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
         for (int rr = lane; rr < 128; rr += 32) {
           const int64_t row = (int64_t)tile * 128 + rr;
           if (row < args.n) {
-            cp_async_8(dst + rr * C::SC_ROW, src + row * ng);
-            cp_async_8(dst + rr * C::SC_ROW + 8, src + row * ng + 4);
+#pragma unroll
+            for (int q8 = 0; q8 < C::SC_ROW / 8; ++q8)  // four scales per 8-byte copy
+              cp_async_8(dst + rr * C::SC_ROW + 8 * q8, src + row * ng + 4 * q8);
           }
         }
       }
@@ -211,9 +212,10 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
         for (int gg = 0; gg < GPP; ++gg) {
           const int gi = h * GPP + gg;  // group within the unit
           uint32_t v[C::ACOLS];
-          // high-bit plane rows are UBS * 32 bytes; dequant_group adds r * 32
+          // second-plane rows are UBS * HROW bytes
           dequant_group<FMT>(st + (gi / Tr::GPB) * BOX_BYTES,
-                             st + C::OFF_HIB + r * 32 * UBS + (gi / Tr::GPB) * 32 - r * 32, r, gi % Tr::GPB, v);
+                             st + C::OFF_HIB + r * Tr::HROW * UBS + (gi / Tr::GPB) * Tr::HROW, r,
+                             gi % Tr::GPB, v);
           float g0[T], g1[T];  // two FMA chains per token
 #pragma unroll
           for (int t = 0; t < T; ++t) g0[t] = g1[t] = 0.0f;
@@ -324,6 +326,8 @@ int unit_k_sm(int fmt) {
   switch (fmt) {
     case QLIN_Q4_G64: return sm_unit_k<QLIN_Q4_G64>();
     case QLIN_Q5_G64: return sm_unit_k<QLIN_Q5_G64>();
+    case QLIN_Q3_G64: return sm_unit_k<QLIN_Q3_G64>();
+    case QLIN_Q6_G64: return sm_unit_k<QLIN_Q6_G64>();
     case QLIN_Q8_G32: return sm_unit_k<QLIN_Q8_G32>();
     case QLIN_FP8_ROW: return sm_unit_k<QLIN_FP8_ROW>();
     default: return sm_unit_k<QLIN_BF16>();
@@ -371,9 +375,7 @@ int launch_gemv_sm(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
   const int64_t cpt = w.k / kc;
   const int64_t units = tiles * cpt;
   const int grid = (int)std::min<int64_t>(ex.num_sms, units);
-  const int64_t row_bytes = w.fmt == QLIN_Q4_G64 || w.fmt == QLIN_Q5_G64 ? w.k / 2
-                            : w.fmt == QLIN_BF16                      ? w.k * 2
-                                                                      : w.k;
+  const int64_t row_bytes = code_row_bytes(w.fmt, w.k);
   CUtensorMap mc, mh, mx;
   int rc = encode_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, (uint64_t)row_bytes,
                           (uint64_t)w.n, (uint64_t)row_bytes, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -381,10 +383,12 @@ int launch_gemv_sm(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
   rc = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)w.k, (uint64_t)t,
                       (uint64_t)w.k * 2, 64, (uint32_t)t, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
-  if (w.fmt == QLIN_Q5_G64) {
-    const uint32_t hib_box = (uint32_t)(32 * (kc / 256));
-    rc = encode_tmap_2d(&mh, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.hibits, (uint64_t)(w.k / 8),
-                        (uint64_t)w.n, (uint64_t)(w.k / 8), hib_box, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (hrow_of(w.fmt) != 0) {
+    // second plane: its bytes for the unit's K columns per row
+    const uint32_t hib_box = (uint32_t)hib_row_bytes(w.fmt, kc);
+    const uint64_t hib_row = (uint64_t)hib_row_bytes(w.fmt, w.k);
+    rc = encode_tmap_2d(&mh, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.hibits, hib_row, (uint64_t)w.n, hib_row,
+                        hib_box, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
   } else {
     mh = mc;
@@ -404,6 +408,8 @@ int launch_gemv_sm(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
   switch (w.fmt) {
     case QLIN_Q4_G64: return launch_fmt_sm<QLIN_Q4_G64>(t, mc, mh, mx, a, grid, ex.stream);
     case QLIN_Q5_G64: return launch_fmt_sm<QLIN_Q5_G64>(t, mc, mh, mx, a, grid, ex.stream);
+    case QLIN_Q3_G64: return launch_fmt_sm<QLIN_Q3_G64>(t, mc, mh, mx, a, grid, ex.stream);
+    case QLIN_Q6_G64: return launch_fmt_sm<QLIN_Q6_G64>(t, mc, mh, mx, a, grid, ex.stream);
     case QLIN_Q8_G32: return launch_fmt_sm<QLIN_Q8_G32>(t, mc, mh, mx, a, grid, ex.stream);
     case QLIN_FP8_ROW: return launch_fmt_sm<QLIN_FP8_ROW>(t, mc, mh, mx, a, grid, ex.stream);
     default: return launch_fmt_sm<QLIN_BF16>(t, mc, mh, mx, a, grid, ex.stream);

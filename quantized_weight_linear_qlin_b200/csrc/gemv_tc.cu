@@ -50,7 +50,7 @@ struct Layout {
   static constexpr int KC = Tr::GK * GPC;             // K columns per unit
   static constexpr int XBOXES = KC / 64;              // activation boxes (64 columns each)
   static constexpr int X_BYTES = XBOXES * TP * 128;
-  static constexpr int HIB_BYTES = Tr::HIB ? UB * 128 * 32 : 0;
+  static constexpr int HIB_BYTES = Tr::HIB ? UB * 128 * Tr::HROW : 0;
   static constexpr int SC_ROW = Tr::PER_GROUP ? GPC * 2 : 0;  // scale bytes per row per unit
   static constexpr int SC_BYTES = 128 * SC_ROW;
   static constexpr int TMA_BYTES = UB * BOX_BYTES + X_BYTES + HIB_BYTES;
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int b = 0; b < UB; ++b)
           tma_load_2d(codes_s + (s * UB + b) * BOX_BYTES, &tm_codes, &full[s], (ch * UB + b) * 128, tile * 128);
-        if (Tr::HIB) tma_load_2d(hib_s + s * L::HIB_BYTES, &tm_hib, &full[s], ch * UB * 32, tile * 128);
+        if (Tr::HIB) tma_load_2d(hib_s + s * L::HIB_BYTES, &tm_hib, &full[s], ch * UB * Tr::HROW, tile * 128);
 #pragma unroll
         for (int b = 0; b < L::XBOXES; ++b)
           tma_load_2d(x_s + s * L::X_BYTES + b * TP * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0);
@@ -212,12 +212,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int rr = lane; rr < 128; rr += 32) {
           const int64_t row = (int64_t)tile * 128 + rr;
           if (row < args.n) {
-            if constexpr (L::SC_ROW == 16) {
-              cp_async_8(dst + rr * 16, src + row * ng);
-              cp_async_8(dst + rr * 16 + 8, src + row * ng + 4);
-            } else {
-              cp_async_8(dst + rr * L::SC_ROW, src + row * ng);
-            }
+#pragma unroll
+            for (int q8 = 0; q8 < L::SC_ROW / 8; ++q8)  // four scales per 8-byte copy
+              cp_async_8(dst + rr * L::SC_ROW + 8 * q8, src + row * ng + 4 * q8);
           }
         }
       }
@@ -284,7 +281,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int g = 0; g < GB; ++g) {
             const int gi = bi * GB + g;  // group within the unit
             uint32_t v[C::ACOLS];
-            dequant_group<FMT>(cs + (gi / Tr::GPB) * BOX_BYTES, hs + r * 32 * UB + (gi / Tr::GPB) * 32 - r * 32,
+            dequant_group<FMT>(cs + (gi / Tr::GPB) * BOX_BYTES, hs + r * Tr::HROW * UB + (gi / Tr::GPB) * Tr::HROW,
                                r, gi % Tr::GPB, v);
             if constexpr (C::ACOLS == 32)
               tmem_st_x32(a_base + lane_ofs + g * C::ACOLS, v);
@@ -490,6 +487,8 @@ int unit_k(int fmt, int tp) {
   switch (fmt) {
     case QLIN_Q4_G64: return unit_k_fmt<QLIN_Q4_G64>(tp);
     case QLIN_Q5_G64: return unit_k_fmt<QLIN_Q5_G64>(tp);
+    case QLIN_Q3_G64: return unit_k_fmt<QLIN_Q3_G64>(tp);
+    case QLIN_Q6_G64: return unit_k_fmt<QLIN_Q6_G64>(tp);
     case QLIN_Q8_G32: return unit_k_fmt<QLIN_Q8_G32>(tp);
     case QLIN_FP8_ROW: return unit_k_fmt<QLIN_FP8_ROW>(tp);
     default: return unit_k_fmt<QLIN_BF16>(tp);
@@ -541,9 +540,7 @@ int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
   const int64_t cpt = w.k / kc;
   const int64_t units = tiles * cpt;
   const int grid = (int)std::min<int64_t>(ex.num_sms, units);
-  const int64_t row_bytes = w.fmt == QLIN_Q4_G64 || w.fmt == QLIN_Q5_G64 ? w.k / 2
-                            : w.fmt == QLIN_BF16                      ? w.k * 2
-                                                                      : w.k;
+  const int64_t row_bytes = code_row_bytes(w.fmt, w.k);
   CUtensorMap mc, mh, mx;
   int rc = encode_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, (uint64_t)row_bytes,
                           (uint64_t)w.n, (uint64_t)row_bytes, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -551,11 +548,12 @@ int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
   rc = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)w.k, (uint64_t)t,
                       (uint64_t)w.k * 2, 64, (uint32_t)tp, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
-  if (w.fmt == QLIN_Q5_G64) {
-    // high-bit plane: 32 bytes per row per 128-byte box of codes
-    const uint32_t hib_box = (uint32_t)(32 * (kc / 256));
-    rc = encode_tmap_2d(&mh, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.hibits, (uint64_t)(w.k / 8),
-                        (uint64_t)w.n, (uint64_t)(w.k / 8), hib_box, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (hrow_of(w.fmt) != 0) {
+    // second plane: its bytes for the unit's K columns per row
+    const uint32_t hib_box = (uint32_t)hib_row_bytes(w.fmt, kc);
+    const uint64_t hib_row = (uint64_t)hib_row_bytes(w.fmt, w.k);
+    rc = encode_tmap_2d(&mh, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.hibits, hib_row, (uint64_t)w.n, hib_row,
+                        hib_box, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
   } else {
     mh = mc;
@@ -576,6 +574,8 @@ int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
   switch (w.fmt) {
     case QLIN_Q4_G64: return launch_fmt<QLIN_Q4_G64>(tp, mc, mh, mx, a, grid, ex.stream);
     case QLIN_Q5_G64: return launch_fmt<QLIN_Q5_G64>(tp, mc, mh, mx, a, grid, ex.stream);
+    case QLIN_Q3_G64: return launch_fmt<QLIN_Q3_G64>(tp, mc, mh, mx, a, grid, ex.stream);
+    case QLIN_Q6_G64: return launch_fmt<QLIN_Q6_G64>(tp, mc, mh, mx, a, grid, ex.stream);
     case QLIN_Q8_G32: return launch_fmt<QLIN_Q8_G32>(tp, mc, mh, mx, a, grid, ex.stream);
     case QLIN_FP8_ROW: return launch_fmt<QLIN_FP8_ROW>(tp, mc, mh, mx, a, grid, ex.stream);
     default: return launch_fmt<QLIN_BF16>(tp, mc, mh, mx, a, grid, ex.stream);

@@ -8,7 +8,8 @@
 // Uncensored FP8 for NInfer", "Conversion and verification" (E4M3 codes with a
 // weight_scale_inv per 128 x 128 block, re-encoded with fp8_row_maxabs);
 // "Qwen3.8-27B for NInfer -- RTX 5080 16 GB", "Quantization profile"
-// (Q4G64_F16S, Q5G64_F16S); "...NVFP4-NInferV3", "What is in the file" (Q8).
+// (Q3G64_F16S, Q4G64_F16S, Q5G64_F16S); "...MXFP8-CRACK", "Caveats" (Q6
+// groupwise); "...NVFP4-NInferV3", "What is in the file" (Q8).
 #include "qlin_internal.cuh"
 
 namespace qlin {
@@ -85,12 +86,19 @@ __device__ __forceinline__ uint32_t warp_or(uint32_t v, int width) {
   return v;
 }
 
-// ---- Q4 / Q5 group-64: one warp per (row, group); lane l owns elements 2l, 2l+1.
+// ---- Q3 / Q4 / Q5 / Q6 group-64: one warp per (row, group); lane l owns
+// elements 2l, 2l+1.  Planes (u = q + 2^(BITS-1)):
+//   nibble plane (Q4, Q5, Q6: bits 0..3 of u): word j = elements 8j..8j+7,
+//     element 8j+2s+o at bits 16o+4s;
+//   crumb plane (Q3: bits 0..1 of u, as the codes; Q6: bits 4..5, as the high
+//     plane): word c = elements 16c..16c+15, element 16c+2s+o at bits 16o+2s;
+//   bit plane (Q5: bit 4, Q3: bit 2): word h = elements 32h..32h+31, element
+//     32h+8jj+2s+o at bit 16o+4jj+s.
 template <int BITS>
-__global__ void pack_q4q5_kernel(Src s, int64_t n, uint8_t* codes, uint8_t* hibits,
-                                 __half* scales) {
-  constexpr float QMAX = BITS == 4 ? 7.0f : 15.0f;
-  constexpr int OFF = BITS == 4 ? 8 : 16;
+__global__ void pack_groupwise64_kernel(Src s, int64_t n, uint8_t* codes, uint8_t* hibits,
+                                        __half* scales) {
+  constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
+  constexpr int OFF = 1 << (BITS - 1);
   const int64_t ng = s.k / 64;
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
@@ -106,23 +114,31 @@ __global__ void pack_q4q5_kernel(Src s, int64_t n, uint8_t* codes, uint8_t* hibi
     q0 = (int)fminf(fmaxf(rintf(__fdiv_rn(v0, sc)), -QMAX - 1.0f), QMAX);
     q1 = (int)fminf(fmaxf(rintf(__fdiv_rn(v1, sc)), -QMAX - 1.0f), QMAX);
   }
-  uint32_t u0 = (uint32_t)(q0 + OFF), u1 = (uint32_t)(q1 + OFF);
-  // nibble word: lanes 4j..4j+3 cover word j; lane's s = lane & 3
-  int sl = lane & 3;
-  uint32_t part = ((u0 & 0xF) << (4 * sl)) | ((u1 & 0xF) << (16 + 4 * sl));
-  uint32_t word = warp_or(part, 4);
-  if (sl == 0) {
-    uint32_t* row = (uint32_t*)(codes + r * (s.k / 2));
-    row[(e0 >> 3)] = word;
-  }
-  if (BITS == 5) {
-    // element e (in group) = 2*lane + o; word h = lane / 16 ; jj = (lane % 16) / 4 ; s = lane % 4
-    int jj = (lane & 15) >> 2;
-    uint32_t hp = (((u0 >> 4) & 1u) << (4 * jj + sl)) | (((u1 >> 4) & 1u) << (16 + 4 * jj + sl));
-    uint32_t hw = warp_or(hp, 16);
-    if ((lane & 15) == 0) {
-      uint32_t* hrow = (uint32_t*)(hibits + r * (s.k / 8));
-      hrow[(e0 >> 5)] = hw;
+  const uint32_t u0 = (uint32_t)(q0 + OFF), u1 = (uint32_t)(q1 + OFF);
+  // the lane's pair inside its nibble word (lanes 4j..4j+3 share word j), its
+  // crumb word (lanes 8c..8c+7) and its bit word (lanes 16h..16h+15)
+  const int sn = lane & 3, sc2 = lane & 7, jj = (lane & 15) >> 2;
+  auto crumb_word = [&](uint32_t f0, uint32_t f1) {
+    return warp_or(((f0 & 3u) << (2 * sc2)) | ((f1 & 3u) << (16 + 2 * sc2)), 8);
+  };
+  auto bit_word = [&](uint32_t b0, uint32_t b1) {
+    return warp_or(((b0 & 1u) << (4 * jj + sn)) | ((b1 & 1u) << (16 + 4 * jj + sn)), 16);
+  };
+  if constexpr (BITS == 3) {
+    const uint32_t cw = crumb_word(u0, u1);
+    if (sc2 == 0) ((uint32_t*)(codes + r * (s.k / 4)))[e0 >> 4] = cw;
+    const uint32_t hw = bit_word(u0 >> 2, u1 >> 2);
+    if ((lane & 15) == 0) ((uint32_t*)(hibits + r * (s.k / 8)))[e0 >> 5] = hw;
+  } else {
+    const uint32_t word = warp_or(((u0 & 0xFu) << (4 * sn)) | ((u1 & 0xFu) << (16 + 4 * sn)), 4);
+    if (sn == 0) ((uint32_t*)(codes + r * (s.k / 2)))[e0 >> 3] = word;
+    if constexpr (BITS == 5) {
+      const uint32_t hw = bit_word(u0 >> 4, u1 >> 4);
+      if ((lane & 15) == 0) ((uint32_t*)(hibits + r * (s.k / 8)))[e0 >> 5] = hw;
+    }
+    if constexpr (BITS == 6) {
+      const uint32_t cw = crumb_word(u0 >> 4, u1 >> 4);
+      if (sc2 == 0) ((uint32_t*)(hibits + r * (s.k / 4)))[e0 >> 4] = cw;
     }
   }
   if (lane == 0) scales[r * ng + g] = s16;
@@ -270,16 +286,21 @@ int launch_pack(int src_kind, const void* src, const void* aux0, const void* aux
   Src s{src_kind, src, aux0, aux1, dst.k};
   const int64_t n = dst.n;
   switch (dst.fmt) {
+    case QLIN_Q3_G64:
     case QLIN_Q4_G64:
-    case QLIN_Q5_G64: {
-      int64_t items = n * (dst.k / 64);
-      int64_t blocks = (items + 7) / 8;
-      if (dst.fmt == QLIN_Q4_G64)
-        pack_q4q5_kernel<4><<<(unsigned)blocks, 256, 0, ex.stream>>>(s, n, (uint8_t*)dst.codes,
-                                                                    nullptr, (__half*)dst.scales);
-      else
-        pack_q4q5_kernel<5><<<(unsigned)blocks, 256, 0, ex.stream>>>(
-            s, n, (uint8_t*)dst.codes, (uint8_t*)dst.hibits, (__half*)dst.scales);
+    case QLIN_Q5_G64:
+    case QLIN_Q6_G64: {
+      const int64_t items = n * (dst.k / 64);
+      const unsigned blocks = (unsigned)((items + 7) / 8);
+      uint8_t* c = (uint8_t*)dst.codes;
+      uint8_t* h = (uint8_t*)dst.hibits;
+      __half* sc = (__half*)dst.scales;
+      switch (dst.fmt) {
+        case QLIN_Q3_G64: pack_groupwise64_kernel<3><<<blocks, 256, 0, ex.stream>>>(s, n, c, h, sc); break;
+        case QLIN_Q4_G64: pack_groupwise64_kernel<4><<<blocks, 256, 0, ex.stream>>>(s, n, c, h, sc); break;
+        case QLIN_Q5_G64: pack_groupwise64_kernel<5><<<blocks, 256, 0, ex.stream>>>(s, n, c, h, sc); break;
+        default: pack_groupwise64_kernel<6><<<blocks, 256, 0, ex.stream>>>(s, n, c, h, sc); break;
+      }
       break;
     }
     case QLIN_Q8_G32: {

@@ -11,34 +11,63 @@ namespace gemv {
 constexpr int BOX_BYTES = 128 * 128;  // one TMA box of codes: 128 rows x 128 bytes
 
 // Per format: K per quantization group, groups per 128-byte box of codes,
-// high-bit plane, per-group scales.
+// second (high-bit) plane and its bytes per row per 128-byte box of codes,
+// per-group scales.
 template <int FMT>
 struct TcT;
 template <>
 struct TcT<QLIN_Q4_G64> {
-  static constexpr int GK = 64, GPB = 4;
+  static constexpr int GK = 64, GPB = 4, HROW = 0;
   static constexpr bool PER_GROUP = true, HIB = false;
 };
 template <>
 struct TcT<QLIN_Q5_G64> {
-  static constexpr int GK = 64, GPB = 4;
+  static constexpr int GK = 64, GPB = 4, HROW = 32;  // one bit per element
+  static constexpr bool PER_GROUP = true, HIB = true;
+};
+template <>
+struct TcT<QLIN_Q3_G64> {
+  static constexpr int GK = 64, GPB = 8, HROW = 64;  // 512 crumbs per box, one bit each
+  static constexpr bool PER_GROUP = true, HIB = true;
+};
+template <>
+struct TcT<QLIN_Q6_G64> {
+  static constexpr int GK = 64, GPB = 4, HROW = 64;  // two bits per element
   static constexpr bool PER_GROUP = true, HIB = true;
 };
 template <>
 struct TcT<QLIN_Q8_G32> {
-  static constexpr int GK = 32, GPB = 4;
+  static constexpr int GK = 32, GPB = 4, HROW = 0;
   static constexpr bool PER_GROUP = true, HIB = false;
 };
 template <>
 struct TcT<QLIN_FP8_ROW> {
-  static constexpr int GK = 64, GPB = 2;
+  static constexpr int GK = 64, GPB = 2, HROW = 0;
   static constexpr bool PER_GROUP = false, HIB = false;  // one scale per row, applied at the end
 };
 template <>
 struct TcT<QLIN_BF16> {
-  static constexpr int GK = 64, GPB = 1;
+  static constexpr int GK = 64, GPB = 1, HROW = 0;
   static constexpr bool PER_GROUP = false, HIB = false;
 };
+
+// Bytes per row of a format's code plane and of its second plane (host side).
+inline int64_t code_row_bytes(int fmt, int64_t k) {
+  switch (fmt) {
+    case QLIN_Q3_G64: return k / 4;
+    case QLIN_Q4_G64:
+    case QLIN_Q5_G64:
+    case QLIN_Q6_G64: return k / 2;
+    case QLIN_BF16: return k * 2;
+    default: return k;  // Q8, FP8
+  }
+}
+inline int64_t hib_row_bytes(int fmt, int64_t k) {
+  return fmt == QLIN_Q6_G64 ? k / 4 : (fmt == QLIN_Q5_G64 || fmt == QLIN_Q3_G64) ? k / 8 : 0;
+}
+inline int hrow_of(int fmt) {
+  return fmt == QLIN_Q5_G64 ? 32 : (fmt == QLIN_Q3_G64 || fmt == QLIN_Q6_G64) ? 64 : 0;
+}
 
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -52,19 +81,26 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
 }
 
 // ---- dequantization of one group of row r into BF16 pairs (element 2c in the
-// low half of v[c]).  `codes` is the 128-byte-swizzled stage tile.
+// low half of v[c]).  `codes` is the 128-byte-swizzled stage tile of the code
+// plane; `hrow` points at row r's bytes of the second plane for this box.
 template <int FMT>
-__device__ __forceinline__ void dequant_group(const uint8_t* codes, const uint8_t* hib, int r, int gi,
+__device__ __forceinline__ void dequant_group(const uint8_t* codes, const uint8_t* hrow, int r, int gi,
                                               uint32_t* v) {
-  if constexpr (FMT == QLIN_Q4_G64 || FMT == QLIN_Q5_G64) {
+  if constexpr (FMT == QLIN_Q4_G64 || FMT == QLIN_Q5_G64 || FMT == QLIN_Q6_G64) {
     const uint4 c0 = *(const uint4*)(codes + sw128_offset(r, 2 * gi));
     const uint4 c1 = *(const uint4*)(codes + sw128_offset(r, 2 * gi + 1));
     const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    uint32_t h0 = 0, h1 = 0;
+    uint32_t h[4] = {0u, 0u, 0u, 0u};
     if constexpr (FMT == QLIN_Q5_G64) {
-      const uint2 hh = *(const uint2*)(hib + r * 32 + gi * 8);
-      h0 = hh.x;
-      h1 = hh.y;
+      const uint2 hh = *(const uint2*)(hrow + gi * 8);  // bit words of elements 0..31, 32..63
+      h[0] = hh.x;
+      h[1] = hh.y;
+    } else if constexpr (FMT == QLIN_Q6_G64) {
+      const uint4 hh = *(const uint4*)(hrow + gi * 16);  // crumb words of elements 16c..16c+15
+      h[0] = hh.x;
+      h[1] = hh.y;
+      h[2] = hh.z;
+      h[3] = hh.w;
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -72,14 +108,37 @@ __device__ __forceinline__ void dequant_group(const uint8_t* codes, const uint8_
       for (int s = 0; s < 4; ++s) {
         uint32_t m = ((w[j] >> (4 * s)) & 0x000F000Fu) | 0x43004300u;  // 128 + u, exact BF16
         if constexpr (FMT == QLIN_Q5_G64) {
-          const uint32_t H = j < 4 ? h0 : h1;
-          const int sh = 4 * (j & 3) + s - 4;  // high bits of the pair -> bits 4 and 20
-          const uint32_t hs = sh >= 0 ? (H >> sh) : (H << (-sh));
-          m |= hs & 0x00100010u;
-          v[4 * j + s] = bf16x2_sub(m, 0x43104310u);  // - 144 = -(128 + 16)
-        } else {
-          v[4 * j + s] = bf16x2_sub(m, 0x43084308u);  // - 136 = -(128 + 8)
+          // bit of element 8j+2s+o at 16o + 4(j&3) + s -> bits 4 and 20
+          const int sh = 4 * (j & 3) + s - 4;
+          const uint32_t H = j < 4 ? h[0] : h[1];
+          m |= (sh >= 0 ? (H >> sh) : (H << (-sh))) & 0x00100010u;
+        } else if constexpr (FMT == QLIN_Q6_G64) {
+          // crumb of element 8j+2s+o: word j/2, bits 16o + 8(j&1) + 2s -> bits 4..5 and 20..21
+          const int sh = 8 * (j & 1) + 2 * s - 4;
+          const uint32_t H = h[j >> 1];
+          m |= (sh >= 0 ? (H >> sh) : (H << (-sh))) & 0x00300030u;
         }
+        v[4 * j + s] = m;
+      }
+    }
+    // 128 + u minus 128 + 2^(bits-1): the signed code, exact
+    constexpr uint32_t OFF = FMT == QLIN_Q4_G64 ? 0x43084308u : FMT == QLIN_Q5_G64 ? 0x43104310u : 0x43204320u;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = bf16x2_sub(v[c], OFF);
+  } else if constexpr (FMT == QLIN_Q3_G64) {
+    const uint4 c = *(const uint4*)(codes + sw128_offset(r, gi));  // crumb words of the group
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    const uint2 hh = *(const uint2*)(hrow + gi * 8);                // bit words
+#pragma unroll
+    for (int cw = 0; cw < 4; ++cw) {
+      const uint32_t H = cw < 2 ? hh.x : hh.y;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        // element 16cw+2s+o: crumb at 16o + 2s; its bit at 16o + 8(cw&1) + 4(s>>2) + (s&3) -> bit 2
+        const int sh = 8 * (cw & 1) + 4 * (s >> 2) + (s & 3) - 2;
+        const uint32_t hs = (sh >= 0 ? (H >> sh) : (H << (-sh))) & 0x00040004u;
+        const uint32_t m = ((w[cw] >> (2 * s)) & 0x00030003u) | hs | 0x43004300u;  // 128 + u
+        v[8 * cw + s] = bf16x2_sub(m, 0x43044304u);                             // - (128 + 4)
       }
     }
   } else if constexpr (FMT == QLIN_Q8_G32) {

@@ -49,12 +49,14 @@ def test_packed_bytes(L):
     assert q.qlin_packed_bytes(q.Q8_G32, 5120, 5120) == (5120 * 5120, 0, 5120 * 160 * 2)
     assert q.qlin_packed_bytes(q.FP8_ROW, 152064, 5120) == (152064 * 5120, 0, 152064 * 2)
     assert q.qlin_packed_bytes(q.BF16, 96, 5120) == (96 * 5120 * 2, 0, 0)
+    assert q.qlin_packed_bytes(q.Q3_G64, 34816, 5120) == (34816 * 1280, 34816 * 640, 34816 * 80 * 2)
+    assert q.qlin_packed_bytes(q.Q6_G64, 5120, 17408) == (5120 * 8704, 5120 * 4352, 5120 * 272 * 2)
     # the configs' algorithmic weight bytes
     c, h, s = q.qlin_packed_bytes(q.Q4_G64, 34816, 5120)
     assert c + h + s == 94_699_520
     c, h, s = q.qlin_packed_bytes(q.Q5_G64, 5120, 17408)
     assert c + h + s == 58_490_880
-    for fmt, k in ((q.Q4_G64, 96), (q.Q8_G32, 48), (7, 64)):
+    for fmt, k in ((q.Q4_G64, 96), (q.Q8_G32, 48), (q.Q3_G64, 96), (q.Q6_G64, 32), (9, 64)):
         with pytest.raises(q.QlinError) as e:
             q.qlin_packed_bytes(fmt, 4, k)
         assert e.value.status == q.ERR_INVALID_ARG
@@ -63,7 +65,7 @@ def test_packed_bytes(L):
 def _weights(fmt, n, k, flags=0, addr=0x10000):
     d = q._Weights()
     d.fmt, d.flags, d.n, d.k = fmt, flags, n, k
-    d.codes, d.hibits, d.scales = addr, addr + 0x1000 if fmt == q.Q5_G64 else None, \
+    d.codes, d.hibits, d.scales = addr, addr + 0x1000 if fmt in (q.Q5_G64, q.Q3_G64, q.Q6_G64) else None, \
         None if fmt == q.BF16 else addr + 0x2000
     return d
 
@@ -87,10 +89,11 @@ def test_host_validation_rejects_before_cuda(L):
     # K not a multiple of the group
     bad = _weights(q.Q4_G64, 256, 96)
     assert L.qlin_gemv(C.byref(bad), fake, 1, fake, q.OUT_BF16, C.byref(ex)) == q.ERR_INVALID_ARG
-    # Q5 needs its high-bit plane
-    w5 = _weights(q.Q5_G64, 256, 512)
-    w5.hibits = None
-    assert L.qlin_gemv(C.byref(w5), fake, 1, fake, q.OUT_BF16, C.byref(ex)) == q.ERR_INVALID_ARG
+    # Q5, Q3 and Q6 need their second plane
+    for fmt in (q.Q5_G64, q.Q3_G64, q.Q6_G64):
+        w5 = _weights(fmt, 256, 512)
+        w5.hibits = None
+        assert L.qlin_gemv(C.byref(w5), fake, 1, fake, q.OUT_BF16, C.byref(ex)) == q.ERR_INVALID_ARG
     # int8 route: permission, formats, activation arguments
     a16 = _weights(q.Q4_G64, 256, 512, flags=0)
     assert L.qlin_gemm_a8(C.byref(a16), fake, None, None, 256, fake, q.OUT_BF16, 0, None,

@@ -14,7 +14,8 @@ import synth
 
 pytestmark = pytest.mark.gpu
 
-FMTS = {"q4": q.Q4_G64, "q5": q.Q5_G64, "q8": q.Q8_G32, "fp8": q.FP8_ROW, "bf16": q.BF16}
+FMTS = {"q4": q.Q4_G64, "q5": q.Q5_G64, "q8": q.Q8_G32, "fp8": q.FP8_ROW, "bf16": q.BF16,
+        "q3": q.Q3_G64, "q6": q.Q6_G64}
 DEV = "cuda"
 
 
@@ -77,7 +78,7 @@ def test_pack_from_f32_bit_exact(fmt, shape):
     assert_packed_equal(pw, ref)
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q5", "q8", "fp8"])
+@pytest.mark.parametrize("fmt", ["q4", "q5", "q8", "fp8", "q3", "q6"])
 def test_pack_from_bf16_bit_exact(fmt):
     w = synth.weights_f32(96, 512, seed=7).to(torch.bfloat16)
     ref = oracle.pack(FMTS[fmt], w.float().numpy())
@@ -86,7 +87,7 @@ def test_pack_from_bf16_bit_exact(fmt):
     assert_packed_equal(pw, ref)
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q5", "q8", "fp8", "bf16"])
+@pytest.mark.parametrize("fmt", ["q4", "q5", "q8", "fp8", "bf16", "q3", "q6"])
 def test_pack_from_mxfp8_bit_exact(fmt):
     rows, cols = 64, 512
     words, scales = synth.mxfp8_source(rows, cols, seed=11)
@@ -231,7 +232,7 @@ def test_gemv_tensor_core_path_split_tiles(fmt, t):
     assert not counters.any()
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q5", "fp8"])
+@pytest.mark.parametrize("fmt", ["q4", "q5", "fp8", "q3", "q6"])
 def test_gemv_bf16_output_and_long_k(fmt):
     n, k, t = 96, 17408, 2
     w = synth.weights_f32(n, k, seed=5)
@@ -261,6 +262,11 @@ def test_gemv_bf16_weights_prefill_sizes(t):
     # the head in both formats at the top of the verify range (FP8-vs-Q8 crossover)
     ("head_q8_T64", q.Q8_G32, 152064, 5120, 64),
     ("head_fp8_T64", q.FP8_ROW, 152064, 5120, 64),
+    # the other group-64 widths at the MLP shapes
+    ("gate_up_q3", q.Q3_G64, 34816, 5120, 1),
+    ("gate_up_q3_T17", q.Q3_G64, 34816, 5120, 17),
+    ("down_q6", q.Q6_G64, 5120, 17408, 33),
+    ("down_q6_T1", q.Q6_G64, 5120, 17408, 1),
 ])
 def test_gemv_full_size_sampled_rows(name, fmt, n, k, t):
     """Full-size weights in the bench's launch configuration; the oracle
@@ -342,7 +348,7 @@ def run_gemm_a8(pw, x, fused=True, debug=True, y_dtype=q.OUT_F32):
     return y, dbg
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q5"])
+@pytest.mark.parametrize("fmt", ["q4", "q5", "q3", "q6"])
 @pytest.mark.parametrize("n,k,t", [(128, 256, 128), (256, 512, 130), (200, 640, 257), (384, 1152, 1),
                                    (128, 5120, 64)])
 def test_gemm_a8_group_sums_bit_exact_and_output(fmt, n, k, t):
@@ -360,7 +366,7 @@ def test_gemm_a8_group_sums_bit_exact_and_output(fmt, n, k, t):
     assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
 
 
-@pytest.mark.parametrize("fmt", ["q4", "q5"])
+@pytest.mark.parametrize("fmt", ["q4", "q5", "q3", "q6"])
 def test_gemm_a8_prequantized_and_bf16_out(fmt):
     n, k, t = 256, 1024, 300
     w = synth.weights_f32(n, k, seed=41)
@@ -372,6 +378,22 @@ def test_gemm_a8_prequantized_and_bf16_out(fmt):
     yr, br = oracle.gemm_a8(ref, qa, as_, nthreads=8)
     got = y.float().cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - yr) <= 5e-6 * br + np.abs(yr) * 2.0 ** -8)
+
+
+@pytest.mark.parametrize("fmt,qmax", [(q.Q3_G64, 3), (q.Q6_G64, 31)])
+def test_gemm_a8_extreme_codes_q3_q6(fmt, qmax):
+    """Every code at +-Qmax against activation codes +-127: |S| = 64 * Qmax * 127, exact."""
+    n, k, t = 128, 512, 128
+    w = torch.full((n, k), 0.5, dtype=torch.float32)
+    w[::2] *= -1
+    x = torch.full((t, k), 2.0, dtype=torch.float32).to(torch.bfloat16)
+    pw = pack_gpu(fmt, w.to(DEV), allow_a8=True)
+    y, dbg = run_gemm_a8(pw, x, fused=True, debug=True)
+    S = dbg.cpu().numpy()
+    assert np.all(np.abs(S) == 64 * qmax * 127)
+    ref = oracle.pack(fmt, w.numpy())
+    qa, as_ = oracle.quantize_act(bits16(x))
+    assert np.array_equal(S, oracle.group_sums(ref, qa))
 
 
 def test_gemm_a8_extreme_codes():
@@ -390,7 +412,9 @@ def test_gemm_a8_extreme_codes():
 
 
 @pytest.mark.parametrize("name,fmt,n,k", [("gate_up_q4", q.Q4_G64, 34816, 5120),
-                                          ("down_q5", q.Q5_G64, 5120, 17408)])
+                                          ("down_q5", q.Q5_G64, 5120, 17408),
+                                          ("gate_up_q3", q.Q3_G64, 34816, 5120),
+                                          ("down_q6", q.Q6_G64, 5120, 17408)])
 def test_gemm_a8_full_size_sampled(name, fmt, n, k):
     t = 2048
     w = synth.weights_f32(n, k, seed=synth.seed_for(3, 0), device=DEV)
@@ -413,7 +437,8 @@ def test_gemm_a8_full_size_sampled(name, fmt, n, k):
 # ---------------------------------------------------------------------------
 # ties: quotients exactly on k + 1/2 (hand-worked groups, tests/golden)
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("name,fmt", [("q4_group", "q4"), ("q5_group", "q5"), ("q8_group", "q8")])
+@pytest.mark.parametrize("name,fmt", [("q4_group", "q4"), ("q5_group", "q5"), ("q8_group", "q8"),
+                                      ("q3_group", "q3"), ("q6_group", "q6")])
 def test_pack_ties_bit_exact(golden, name, fmt):
     ex = golden["ties"][name]
     gs = 32 if fmt == "q8" else 64
