@@ -51,8 +51,8 @@ def parse():
     p.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     p.add_argument("--case", default=None,
-                   help="run one kernel case only (for profilers): gemv:<q4|q5|q8|fp8|bf16>:<N>x<K>:T<t> "
-                        "or gemm_a8:<q4|q5>:<N>x<K>:T<t> or quantize:<T>x<K> or decode:<R>x<C>")
+                   help="run one kernel case only (for profilers): gemv:<q3|q4|q5|q6|q8|fp8|bf16>:<N>x<K>:T<t> "
+                        "or gemm_a8:<q3|q4|q5|q6>:<N>x<K>:T<t> or quantize:<T>x<K> or decode:<R>x<C>")
     return p.parse_args()
 
 
@@ -496,6 +496,20 @@ def measure_rows(ctx):
             res[f"T={t}"] = {"us": round(ms * 1e3, 1), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
                               "frac_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 3)}
         rows[name] = res
+    # the Q3 / Q6 group-64 widths at the MLP shapes (decode GEMV)
+    for name, fmt, (n, k) in (("gemv_q3_gate_up", q.Q3_G64, GATE_UP), ("gemv_q6_down", q.Q6_G64, DOWN)):
+        pw = packed(q, synth, fmt, n, k, 16, dev, allow_a8=True)
+        res = {}
+        for t in T_LIST:
+            x = synth.activations_bf16(t, k, seed=5, device=dev)
+            y = torch.empty(t, n, dtype=torch.bfloat16, device=dev)
+            ws.ensure(q.qlin_gemv_workspace_bytes(pw, t))
+            ms = time_fn(lambda: q.qlin_gemv(pw, x, y, q.OUT_BF16, workspace=ws), flush=flush)
+            gbs = gemv_bytes(pw, t) / ms / 1e6
+            res[f"T={t}"] = {"us": round(ms * 1e3, 1), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                             "frac_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 3)}
+        rows[name] = res
+        del pw
     # activation quantizer, T=2048 x 17408
     x = synth.activations_bf16(2048, 17408, seed=6, device=dev)
     xq = torch.empty(2048, 17408, dtype=torch.int8, device=dev)
@@ -519,7 +533,8 @@ def measure_rows(ctx):
     peak = int8_peak or 4500.0
     # int8 prefill GEMM, 2048 tokens (fused quantizer)
     res = {}
-    for name, fmt, (n, k) in (("gate_up_q4", q.Q4_G64, GATE_UP), ("down_q5", q.Q5_G64, DOWN)):
+    for name, fmt, (n, k) in (("gate_up_q4", q.Q4_G64, GATE_UP), ("down_q5", q.Q5_G64, DOWN),
+                              ("gate_up_q3", q.Q3_G64, GATE_UP), ("down_q6", q.Q6_G64, DOWN)):
         pw = packed(q, synth, fmt, n, k, 7, dev, allow_a8=True)
         x = synth.activations_bf16(2048, k, seed=8, device=dev)
         y = torch.empty(2048, n, dtype=torch.bfloat16, device=dev)
@@ -554,7 +569,9 @@ def measure_rows(ctx):
         sweep[f"T={t}"] = {"ms": round(ms, 3), "TOPS": round(ops / ms / 1e9, 1),
                            "frac_int8_peak": round(ops / ms / 1e9 / peak, 3),
                            "tok_per_s_linear_only": round(t / ms * 1e3, 1),
-                           "gdn_ab_bf16_us": round(gms * 1e3, 1)}
+                           "gdn_ab_bf16_us": round(gms * 1e3, 1),
+                           "gdn_ab_GB/s": round((t * 5120 * 2 + 96 * 5120 * 2 + t * 96 * 2) / gms / 1e6, 1),
+                           "gdn_ab_frac_hbm": round((t * 5120 * 2 + 96 * 5120 * 2 + t * 96 * 2) / gms / 1e6 / hbm, 3)}
     rows["prefill_layer_sweep"] = sweep
     del pws, gdn
     rows.update(measure_fp8_route(ctx, flush))
@@ -656,7 +673,8 @@ def run_case(args):
     from quantized_weight_linear_qlin_b200 import _build
     _build.build()
     dev = torch.device("cuda", 0)
-    fmts = {"q4": q.Q4_G64, "q5": q.Q5_G64, "q8": q.Q8_G32, "fp8": q.FP8_ROW, "bf16": q.BF16}
+    fmts = {"q4": q.Q4_G64, "q5": q.Q5_G64, "q8": q.Q8_G32, "fp8": q.FP8_ROW, "bf16": q.BF16,
+            "q3": q.Q3_G64, "q6": q.Q6_G64}
     parts = args.case.split(":")
     kind = parts[0]
     ws = q.Workspace(dev)

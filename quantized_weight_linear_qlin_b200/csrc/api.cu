@@ -20,6 +20,10 @@ int launch_gemv_sm(const qlin_weights& w, const uint16_t* x, int64_t t, void* y,
 size_t gemv_tc_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
 int launch_gemv_tc(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                    const Exec& ex);
+bool gemm_bf16_tok_supported(const qlin_weights& w, int64_t t);
+size_t gemm_bf16_tok_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
+int launch_gemm_bf16_tok(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
+                         const Exec& ex);
 bool gemv_f16_supported(const qlin_weights& w, int64_t t);
 size_t gemv_f16_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
 int launch_gemv_f16(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
@@ -170,8 +174,10 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
 //    2 <= T <= 64 on gemv_tc (exact BF16 integer codes, one FP32 sum per
 //    group scaled in the epilogue): the nibble expansion of gemv_f16 costs
 //    about 13 instructions per 32-bit word, which made it slower there;
-//  - BF16 weights: gemv_tc, in 64-token chunks above 64 tokens (the GDN a/b
-//    projection at prefill; the weights, 1 MB for 96 x 5120, stay in L2);
+//  - BF16 weights: gemv_tc up to 64 tokens; above that, with N <= 256 (the
+//    GDN a/b projection at prefill), gemm_bf16_tok: tokens on the MMA's M
+//    side, K split over CTAs until every SM streams a share of x; larger N in
+//    64-token gemv_tc chunks;
 //  - rows that are not whole units: the CUDA-core kernel.
 constexpr int64_t kTcMaxT = 64;
 static bool bf16_chunked(const qlin_weights& w, int64_t t) {
@@ -183,6 +189,7 @@ static bool use_f16(const qlin_weights& w, int64_t t) {
 }
 
 size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
+  if (gemm_bf16_tok_supported(w, t)) return gemm_bf16_tok_workspace_bytes(w, t, num_sms);
   if (use_f16(w, t)) return gemv_f16_workspace_bytes(w, t, num_sms);
   if (gemv_sm_supported(w, t)) return gemv_sm_workspace_bytes(w, t, num_sms);
   if (bf16_chunked(w, t)) return gemv_tc_workspace_bytes(w, kTcMaxT, num_sms);
@@ -192,6 +199,7 @@ size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
 
 int launch_gemv(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                 const Exec& ex) {
+  if (gemm_bf16_tok_supported(w, t)) return launch_gemm_bf16_tok(w, x, t, y, y_dtype, ex);
   if (use_f16(w, t)) return launch_gemv_f16(w, x, t, y, y_dtype, ex);
   if (gemv_sm_supported(w, t)) return launch_gemv_sm(w, x, t, y, y_dtype, ex);
   if (bf16_chunked(w, t)) {

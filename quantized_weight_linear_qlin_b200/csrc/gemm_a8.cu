@@ -5,8 +5,11 @@
 // activation_scale in FP32.
 //
 // B200 design:
-//   * quantize_act_kernel: eight lanes per (token, 64-group), 16-byte loads;
-//     amax by shuffles, IEEE division, RNE.
+//   * quantize_act_kernel: eight lanes per (token, 64-group), 16-byte loads
+//     (two per thread in flight); amax by shuffles, the scale by IEEE
+//     division, the codes rint(x / scale) through the correctly rounded
+//     reciprocal with the IEEE division taking over near a half-integer
+//     (bit-identical to one division per element, see rint_quot).
 //   * gemm_a8_kernel: persistent, one CTA per SM walking 128-row x 128-token
 //     tiles (neighbouring CTAs share weight rows; the activations stay in L2):
 //       - a TMA warp streams the packed weight codes, the int8 activation codes
@@ -38,45 +41,68 @@ namespace {
 // Eight lanes per 64-group (8 elements = 16 bytes each), four groups per warp;
 // x is [T][K] with K % 64 == 0, so group g covers elements [64g, 64g + 64) of
 // the flattened array and its scale is xs[g].
-__global__ void quantize_act_kernel(const uint16_t* __restrict__ x, int64_t groups,
-                                    int8_t* __restrict__ xq, float* __restrict__ xs) {
+// rint(x / sc) in FP32 without a division per element: with rc = 1/sc
+// correctly rounded, t = x * rc differs from the exact quotient Q by at most
+// 2^-23 |Q| <= 2^-16 (|Q| <= 127.5), and the IEEE quotient fl(Q) by at most
+// 2^-24 |Q|.  So unless t lies within 2^-13 of a half-integer, rint(t) and
+// rint(fl(Q)) are the same integer; near a half-integer (exact ties included)
+// the IEEE division decides.  Any inf / NaN on the way (a subnormal scale
+// whose reciprocal overflows, non-finite inputs) also takes the division.
+__device__ __forceinline__ float rint_quot(float x, float sc, float rc) {
+  const float t = x * rc;
+  const float d = fabsf((t - floorf(t)) - 0.5f);
+  return d > 0x1p-13f ? rintf(t) : rintf(__fdiv_rn(x, sc));
+}
+
+__device__ __forceinline__ void quantize_group8(uint4 raw, int lane, bool valid, int64_t idx,
+                                                int8_t* __restrict__ xq, float* __restrict__ xs) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+  // the 8 lanes of a group are consecutive and aligned to 8 within the warp
+#pragma unroll
+  for (int o = 4; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  const float sc = __fdiv_rn(a, 127.0f);
+  uint32_t packed[2] = {0u, 0u};
+  if (sc != 0.0f) {
+    const float rc = __frcp_rn(sc);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int q = (int)fminf(fmaxf(rint_quot(v[i], sc, rc), -127.0f), 127.0f);
+      packed[i >> 2] |= ((uint32_t)q & 0xFFu) << (8 * (i & 3));
+    }
+  }
+  if (valid) {
+    __stcg((uint2*)(xq + idx * 8), make_uint2(packed[0], packed[1]));
+    if ((lane & 7) == 0) xs[idx >> 3] = sc;
+  }
+}
+
+__global__ void __launch_bounds__(512) quantize_act_kernel(const uint16_t* __restrict__ x, int64_t groups,
+                                                           int8_t* __restrict__ xq, float* __restrict__ xs) {
   // let the GEMM that consumes these codes start its prologue now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t total = groups * 8;  // 8 lanes per group
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  // whole warps iterate together (the shuffles need every lane)
-  for (int64_t wbase = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); wbase < total; wbase += stride) {
-    const int64_t idx = wbase + lane;
-    const bool valid = idx < total;  // total % 8 == 0: a group is valid or not as a whole
-    const int64_t e0 = idx * 8;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (valid) raw = __ldcs((const uint4*)(x + e0));
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-    float a = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
-    // the 8 lanes of a group are consecutive and aligned to 8 within the warp
-#pragma unroll
-    for (int o = 4; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const float sc = __fdiv_rn(a, 127.0f);
-    uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      int q = 0;
-      if (sc != 0.0f) q = (int)fminf(fmaxf(rintf(__fdiv_rn(v[i], sc)), -127.0f), 127.0f);
-      packed[i >> 2] |= ((uint32_t)q & 0xFFu) << (8 * (i & 3));
-    }
-    if (valid) {
-      __stcg((uint2*)(xq + e0), make_uint2(packed[0], packed[1]));
-      if ((lane & 7) == 0) xs[idx >> 3] = sc;
-    }
+  // whole warps iterate together (the shuffles need every lane); two 16-byte
+  // loads per thread in flight
+  for (int64_t wbase = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); wbase < total;
+       wbase += 2 * stride) {
+    const int64_t i0 = wbase + lane, i1 = wbase + stride + lane;
+    const bool v0 = i0 < total, v1 = i1 < total;  // total % 8 == 0: a group is valid or not as a whole
+    uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
+    if (v0) r0 = __ldcs((const uint4*)(x + i0 * 8));
+    if (v1) r1 = __ldcs((const uint4*)(x + i1 * 8));
+    quantize_group8(r0, lane, v0, i0, xq, xs);
+    if (__any_sync(0xffffffffu, v1)) quantize_group8(r1, lane, v1, i1, xq, xs);
   }
 }
 

@@ -242,16 +242,55 @@ def test_gemv_bf16_output_and_long_k(fmt):
     check_gemv(pw, ref, x, q.OUT_BF16)
 
 
-@pytest.mark.parametrize("t", [130, 512])
+@pytest.mark.parametrize("t", [65, 130, 512, 1792])
 def test_gemv_bf16_weights_prefill_sizes(t):
-    # GDN a/b projection kept in BF16: 96 x 5120 at a prefill chunk (64-token
-    # tensor-core launches; 130 leaves a ragged last chunk)
+    # GDN a/b projection kept in BF16: 96 x 5120 at a prefill chunk (tokens on
+    # the MMA's M side, K split over CTAs; 65 and 130 leave ragged token tiles)
     n, k = 96, 5120
     w = synth.weights_f32(n, k, seed=9)
     x = synth.activations_bf16(t, k, seed=10)
     ref = oracle.pack(q.BF16, w.numpy())
     pw = pack_gpu(q.BF16, w.to(DEV))
     check_gemv(pw, ref, x, q.OUT_F32)
+
+
+@pytest.mark.parametrize("n,k,t,y_dtype", [(80, 1024, 300, q.OUT_BF16), (256, 640, 129, q.OUT_F32),
+                                           (16, 4096, 2000, q.OUT_F32), (200, 192, 777, q.OUT_BF16),
+                                           (96, 5120, 1100, q.OUT_BF16), (64, 2048, 1025, q.OUT_F32)])
+def test_gemv_bf16_weights_prefill_ragged_n(n, k, t, y_dtype):
+    """Small BF16 projections at prefill sizes: N padded inside the kernel
+    (80 -> 96, 200 -> 256), few K stages (K = 192: one part), BF16 and FP32 out;
+    1100 and 1025 tokens leave the last CTA's second 128-token sub-tile wholly
+    or all but one token out of range."""
+    w = synth.weights_f32(n, k, seed=11 + n)
+    x = synth.activations_bf16(t, k, seed=12 + t)
+    ref = oracle.pack(q.BF16, w.numpy())
+    pw = pack_gpu(q.BF16, w.to(DEV))
+    check_gemv(pw, ref, x, y_dtype)
+
+
+@pytest.mark.parametrize("t", [8192, 40000])
+def test_gemv_bf16_gdn_ab_full_size_sampled(t):
+    """The GDN a/b projection 96 x 5120 at an 8192-token prefill chunk (K split
+    three ways) and at 40000 tokens (one part per tile): sampled tokens,
+    always the first and the last (ragged) tile."""
+    n, k = 96, 5120
+    w = synth.weights_f32(n, k, seed=synth.seed_for(5, 0), device=DEV)
+    x = synth.activations_bf16(t, k, seed=synth.seed_for(5, 1), device=DEV)
+    pw = pack_gpu(q.BF16, w)
+    y = torch.empty(t, n, dtype=torch.float32, device=DEV)
+    ws = q.Workspace(DEV).ensure(q.qlin_gemv_workspace_bytes(pw, t))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q.qlin_gemv(pw, x, y, q.OUT_F32, workspace=ws, dev_status=status)
+    g = torch.Generator().manual_seed(t)
+    toks = torch.cat([torch.randperm(t, generator=g)[:40], torch.tensor([0, 127, 128, t - 1])]).unique()
+    ref = oracle.pack(q.BF16, w.cpu().numpy())
+    yr, br = oracle.gemv(ref, bits16(x[toks.to(DEV)]), nthreads=8)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    got = y[toks.to(DEV)].cpu().numpy().astype(np.float64)
+    bad = np.abs(got - yr) > 1e-3 * br
+    assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], yr[bad][:5])
 
 
 @pytest.mark.parametrize("name,fmt,n,k,t", [
