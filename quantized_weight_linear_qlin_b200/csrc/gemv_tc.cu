@@ -20,11 +20,13 @@
 //               owns one weight row, expands the batch's codes to exact BF16
 //               integers (exponent-bias tricks, no conversions) and writes them
 //               with tcgen05.st as the MMA's A operand straight into tensor
-//               memory; after a warpgroup barrier one elected thread issues the
-//               batch's tcgen05.mma.kind::f16 (A in tensor memory, B = the
+//               memory, then each warp arrives on the warpgroup's barrier and
+//               goes on to its next batch;
+//   warps 1-2   issuer w waits for warpgroup w's batch and one elected thread
+//               issues its tcgen05.mma.kind::f16 (A in tensor memory, B = the
 //               activations in shared memory, M = 128, N = T padded to 16), one
-//               FP32 accumulator per group, and commits once.  Two issuing
-//               threads: one thread issues an MMA only every ~65 cycles;
+//               FP32 accumulator per group, and commits once (the expanding
+//               warps no longer stop to issue MMAs themselves);
 //   warpgroup 3 the epilogue reads a batch's 128 x T sums with tcgen05.ld,
 //               applies each group's FP16 scale in FP32 registers and re-zeroes
 //               the accumulators (every MMA accumulates: one that overwrites its
@@ -125,7 +127,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* empty = full + NS;
   uint64_t* d_full = empty + NS;        // [NWG][2], slots 0..NDW-1 used
   uint64_t* d_empty = d_full + 2 * NWG; // [NWG][2]
-  uint32_t* tmem_slot = (uint32_t*)(d_empty + 2 * NWG);
+  uint64_t* a_full = d_empty + 2 * NWG;  // [NWG]: a batch's A operand is written
+  uint32_t* tmem_slot = (uint32_t*)(a_full + NWG);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   volatile int* fix_slot = (volatile int*)(tmem_slot + 2);
 
@@ -145,9 +148,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&empty[s], 128);    // every epilogue thread, once done with the unit's scales
     }
     for (int i = 0; i < 2 * NWG; ++i) {
-      mbar_init(&d_full[i], C::GB);  // one tcgen05.commit per issuing warp
+      mbar_init(&d_full[i], 1);  // the issuer's tcgen05.commit
       mbar_init(&d_empty[i], 128);
     }
+    for (int i = 0; i < NWG; ++i) mbar_init(&a_full[i], 4);  // the warpgroup's four warps
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -229,15 +233,67 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0)
       for (int cu = issued > NS ? issued - NS : 0; cu < issued; ++cu)
         mbar_wait(&full[cu % NS], (uint32_t)((cu / NS) & 1));
+  } else if (warp >= 1 && warp <= NWG) {
+    // ---- MMA issue for warpgroup wg = warp - 1: once the warpgroup's four
+    // warps have written a batch's A operand, one elected thread issues the
+    // batch's MMAs (every group into its own accumulator) and commits once.
+    const int wg = warp - 1;
+    const uint32_t idesc = idesc_bf16(128, TP);
+    const uint32_t a_base = tmem + wg * C::WG_COLS;
+    const uint32_t d_base = a_base + C::A_COLS;
+    bool ok = true;
+    Ring ring{0, 0};
+    Ring dr{0, 0};
+    uint32_t nb = 0;  // batches of this warpgroup so far
+    int bw = 0;       // owner of the next batch
+    for (int cu = 0; cu < nunits && ok; ++cu) {
+      const int s = ring.slot;
+      bool mine = false;
+      {
+        int w = bw;
+        for (int bi = 0; bi < BPU; ++bi) {
+          mine |= w == wg;
+          w = (w + 1 == NWG) ? 0 : w + 1;
+        }
+      }
+      // the stage's activations have landed
+      if (mine) ok = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&full[s], (uint32_t)ring.phase));
+      const uint32_t xs_base = smem_u32(x_s + s * L::X_BYTES);
+      for (int bi = 0; bi < BPU && ok; ++bi, bw = (bw + 1 == NWG) ? 0 : bw + 1) {
+        if (bw != wg) continue;
+        const int ds = dr.slot;
+        // the batch's A operand is written; the accumulator slot was read and
+        // re-zeroed by the epilogue
+        ok = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&a_full[wg], nb & 1u) &&
+                                         mbar_wait(&d_empty[wg * 2 + ds], (uint32_t)(dr.phase ^ 1)));
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int g = 0; g < GB; ++g) {
+            const int kofs = (bi * GB + g) * Tr::GK;  // K offset of the group inside the unit
+            const uint32_t xaddr = xs_base + (kofs / 64) * TP * 128 + (kofs % 64) * 2;
+#pragma unroll
+            for (int kk = 0; kk < Tr::GK / 16; ++kk)
+              mma_f16_ts(d_base + ds * C::D_COLS + g * TP, a_base + g * C::ACOLS + kk * 8,
+                         sdesc_k_sw128(xaddr + kk * 32), idesc, 1u);
+          }
+          tc_commit(&d_full[wg * 2 + ds]);
+        }
+        __syncwarp();
+        ++nb;
+        dr.next(C::NDW);
+      }
+      ring.next(NS);
+    }
+    if (!ok && lane == 0) abort_now();
   } else if (warp >= W_DQ0 && warp < W_EPI0) {
-    // ---- dequantize + issue: warpgroup wg takes the batches b with b % NWG == wg
+    // ---- dequantize: warpgroup wg takes the batches b with b % NWG == wg
     const int wg = (warp - W_DQ0) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_ofs = (uint32_t)(quarter * 32) << 16;
-    const uint32_t idesc = idesc_bf16(128, TP);
     const uint32_t a_base = tmem + wg * C::WG_COLS;
-    const uint32_t d_base = a_base + C::A_COLS;
     bool dead = false;  // after a timed-out wait: skip work, keep the barrier sequence
     Ring ring{0, 0};
     Ring dr{0, 0};       // this warpgroup's accumulator slot
@@ -260,7 +316,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const uint8_t* cs = codes_s + s * UB * BOX_BYTES;
       const uint8_t* hs = hib_s + s * L::HIB_BYTES;
-      const uint32_t xs_base = smem_u32(x_s + s * L::X_BYTES);
       for (int bi = 0; bi < BPU; ++bi, bw = (bw + 1 == NWG) ? 0 : bw + 1) {
         if (bw != wg) continue;
         const int ds = dr.slot;
@@ -290,28 +345,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           tmem_st_wait();
         }
+        // hand the batch to the warpgroup's issuing warp; the four warps never
+        // wait for one another or for the MMA issue
         tc_fence_before();
-        named_barrier_sync(1 + wg, 128);
-        // warp q issues group q of the batch from lane 0: one thread issues an
-        // MMA only every ~45-80 cycles, threads of different warps in parallel
-        bool go = quarter < GB && lane == 0 && !dead;
-        // the accumulator slot was read and re-zeroed by the epilogue (each
-        // issuing thread waits for every use of its warpgroup's slots in order)
-        if (go && !mbar_wait(&d_empty[wg * 2 + ds], (uint32_t)(dr.phase ^ 1))) {
-          go = false;
-          abort_now();
-        }
-        if (go) {
-          tc_fence_after();
-          const int g = quarter;
-          const int kofs = (bi * GB + g) * Tr::GK;  // K offset of the group inside the unit
-          const uint32_t xaddr = xs_base + (kofs / 64) * TP * 128 + (kofs % 64) * 2;
-#pragma unroll
-          for (int kk = 0; kk < Tr::GK / 16; ++kk)
-            mma_f16_ts(d_base + ds * C::D_COLS + g * TP, a_base + g * C::ACOLS + kk * 8,
-                       sdesc_k_sw128(xaddr + kk * 32), idesc, 1u);
-          tc_commit(&d_full[wg * 2 + ds]);
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[wg]);
         prev_slot = ds;
         prev_phase = dr.phase;
         dr.next(C::NDW);
@@ -463,9 +501,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
+  // Every accumulator's completion was observed by the epilogue before this
+  // point -- unless a wait timed out; then give the tensor core ample time
+  // (1 ms) before the tensor memory is released.
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    if (*abort_flag) {
+      const unsigned long long t0 = global_ns();
+      while (global_ns() - t0 < 1000000ull) {
+      }
+    }
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
