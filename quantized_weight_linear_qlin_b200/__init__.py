@@ -104,14 +104,17 @@ def _ptr(t):
         raise ValueError("qlin works on CUDA tensors only (no CPU path)")
     if not t.is_contiguous():
         raise ValueError("qlin needs contiguous tensors")
-    return C.c_void_p(t.data_ptr())
+    return t.data_ptr()
+
+
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_get_device = getattr(torch._C, "_cuda_getDevice", None)
 
 
 def _current_stream_handle():
     """cudaStream_t of torch's current stream on the current device."""
-    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
-    if raw is not None:
-        return raw(torch.cuda.current_device())
+    if _raw_stream is not None and _get_device is not None:
+        return _raw_stream(_get_device())
     return torch.cuda.current_stream().cuda_stream
 
 
