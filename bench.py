@@ -338,15 +338,18 @@ def run_ours(args, dist):
     # launches of our kernels in one step, counted by the CUDA profiler
     launches = count_our_launches(lambda: step(0)) * args.steps
 
-    # ---- e2e: through the public API with pinned host buffers.  The step's
-    # eight activation tensors arrive in one host-to-device copy and the eight
-    # results leave in one device-to-host copy (same bytes as per-call copies).
+    # ---- e2e: through the public API with pinned host buffers.  Each step's
+    # eight activation tensors go up in one host-to-device copy and its eight
+    # results come back in one device-to-host copy, on a copy stream: the
+    # inputs of step i+1 (double-buffered) and the results of step i move while
+    # step i+1 computes, as a serving loop would overlap them.
     xs_list = [x for t in T_LIST for x in (xs_gu[t], xs_dn[t])]
     ys_list = [y for t in T_LIST for y in (ys_gu[t], ys_dn[t])]
     hx_all = torch.cat([x.reshape(-1) for x in xs_list]).cpu().pin_memory()
-    dx_all = torch.empty_like(hx_all, device=dev)
-    dy_all = torch.empty(sum(y.numel() for y in ys_list), dtype=torch.bfloat16, device=dev)
-    hy_all = torch.empty(dy_all.numel(), dtype=torch.bfloat16).pin_memory()
+    n_y = sum(y.numel() for y in ys_list)
+    dx_all = [torch.empty_like(hx_all, device=dev) for _ in range(2)]
+    dy_all = [torch.empty(n_y, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    hy_all = torch.empty(n_y, dtype=torch.bfloat16).pin_memory()
 
     def views(flat, shapes):
         out, o = [], 0
@@ -355,27 +358,43 @@ def run_ours(args, dist):
             out.append(flat[o:o + n].view(shp))
             o += n
         return out
-    dxv = views(dx_all, [tuple(x.shape) for x in xs_list])
-    dyv = views(dy_all, [tuple(y.shape) for y in ys_list])
+    dxv = [views(b, [tuple(x.shape) for x in xs_list]) for b in dx_all]
+    dyv = [views(b, [tuple(y.shape) for y in ys_list]) for b in dy_all]
     h2d = hx_all.numel() * 2
     d2h = hy_all.numel() * 2
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(i):
-        dx_all.copy_(hx_all, non_blocking=True)
-        for ti, t in enumerate(T_LIST):
-            gu, dn = copies[ti]
-            q.qlin_gemv(gu, dxv[2 * ti], dyv[2 * ti], q.OUT_BF16, workspace=ws)
-            q.qlin_gemv(dn, dxv[2 * ti + 1], dyv[2 * ti + 1], q.OUT_BF16, workspace=ws)
-        hy_all.copy_(dy_all, non_blocking=True)
+    def e2e_run(n):
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            dx_all[0].copy_(hx_all, non_blocking=True)
+        h2d_done[0].record(side)
+        for i in range(n):
+            b = i & 1
+            main.wait_event(h2d_done[b])
+            for ti, t in enumerate(T_LIST):
+                gu, dn = copies[ti]
+                q.qlin_gemv(gu, dxv[b][2 * ti], dyv[b][2 * ti], q.OUT_BF16, workspace=ws)
+                q.qlin_gemv(dn, dxv[b][2 * ti + 1], dyv[b][2 * ti + 1], q.OUT_BF16, workspace=ws)
+            comp_done[b].record(main)
+            side.wait_event(comp_done[b])  # step i's results, and its input buffer is free
+            with torch.cuda.stream(side):
+                hy_all.copy_(dy_all[b], non_blocking=True)
+                if i + 1 < n:
+                    dx_all[1 - b].copy_(hx_all, non_blocking=True)
+            if i + 1 < n:
+                h2d_done[1 - b].record(side)
+        main.wait_stream(side)
 
-    for i in range(args.warmup):
-        e2e_step(i)
+    e2e_run(args.warmup)
     torch.cuda.synchronize()
     dist.barrier()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s2.record()
-    for i in range(args.steps):
-        e2e_step(i)
+    e2e_run(args.steps)
     e2.record()
     torch.cuda.synchronize()
     e2e_ms = dist.max(s2.elapsed_time(e2))
