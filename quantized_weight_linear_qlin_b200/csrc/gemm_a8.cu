@@ -9,7 +9,7 @@
 //     (two per thread in flight); amax by shuffles, the scale by IEEE
 //     division, the codes rint(x / scale) through the correctly rounded
 //     reciprocal with the IEEE division taking over near a half-integer
-//     (bit-identical to one division per element, see rint_quot).
+//     (bit-identical to one division per element, see code_fast).
 //   * gemm_a8_kernel: persistent, one CTA per SM walking 128-row x 128-token
 //     tiles (neighbouring CTAs share weight rows; the activations stay in L2):
 //       - a TMA warp streams the packed weight codes, the int8 activation codes
@@ -44,14 +44,25 @@ namespace {
 // rint(x / sc) in FP32 without a division per element: with rc = 1/sc
 // correctly rounded, t = x * rc differs from the exact quotient Q by at most
 // 2^-23 |Q| <= 2^-16 (|Q| <= 127.5), and the IEEE quotient fl(Q) by at most
-// 2^-24 |Q|.  So unless t lies within 2^-13 of a half-integer, rint(t) and
-// rint(fl(Q)) are the same integer; near a half-integer (exact ties included)
-// the IEEE division decides.  Any inf / NaN on the way (a subnormal scale
-// whose reciprocal overflows, non-finite inputs) also takes the division.
-__device__ __forceinline__ float rint_quot(float x, float sc, float rc) {
+// 2^-24 |Q|.  So when t lies farther than 2^-13 from every half-integer,
+// rint(t) and rint(fl(Q)) are the same integer; near a half-integer (exact
+// ties included) the IEEE division decides.  rint(t) comes from one FP32 add
+// of 1.5 * 2^23: the sum's ulp is 1, so it rounds t to the nearest integer
+// (ties to even), the integer sits in the low bits of the sum's bit pattern
+// (its low byte is the int8 code), and t minus it is exact.  Any inf / NaN on
+// the way (a subnormal scale whose reciprocal overflows, non-finite inputs)
+// fails the distance test and also takes the division.
+constexpr float RND_MAGIC = 12582912.0f;  // 1.5 * 2^23
+
+// int8 code byte of x, or -1 when the IEEE division must decide
+__device__ __forceinline__ int code_fast(float x, float rc) {
   const float t = x * rc;
-  const float d = fabsf((t - floorf(t)) - 0.5f);
-  return d > 0x1p-13f ? rintf(t) : rintf(__fdiv_rn(x, sc));
+  const float m = t + RND_MAGIC;
+  const float r = t - (m - RND_MAGIC);
+  return fabsf(r) <= 0.5f - 0x1p-13f ? (int)(__float_as_uint(m) & 0xFFu) : -1;
+}
+__device__ __forceinline__ int code_div(float x, float sc) {
+  return ((int)fminf(fmaxf(rintf(__fdiv_rn(x, sc)), -127.0f), 127.0f)) & 0xFF;
 }
 
 __device__ __forceinline__ void quantize_group8(uint4 raw, int lane, bool valid, int64_t idx,
@@ -73,11 +84,20 @@ __device__ __forceinline__ void quantize_group8(uint4 raw, int lane, bool valid,
   uint32_t packed[2] = {0u, 0u};
   if (sc != 0.0f) {
     const float rc = __frcp_rn(sc);
+    int c[8];
+    bool slow = false;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int q = (int)fminf(fmaxf(rint_quot(v[i], sc, rc), -127.0f), 127.0f);
-      packed[i >> 2] |= ((uint32_t)q & 0xFFu) << (8 * (i & 3));
+      c[i] = code_fast(v[i], rc);
+      slow |= c[i] < 0;
     }
+    if (slow) {  // rare: a code near a half-integer (or a non-finite value)
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (c[i] < 0) c[i] = code_div(v[i], sc);
+    }
+    packed[0] = (uint32_t)c[0] | ((uint32_t)c[1] << 8) | ((uint32_t)c[2] << 16) | ((uint32_t)c[3] << 24);
+    packed[1] = (uint32_t)c[4] | ((uint32_t)c[5] << 8) | ((uint32_t)c[6] << 16) | ((uint32_t)c[7] << 24);
   }
   if (valid) {
     __stcg((uint2*)(xq + idx * 8), make_uint2(packed[0], packed[1]));
