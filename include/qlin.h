@@ -208,7 +208,12 @@ QLIN_API int qlin_gemv_workspace_bytes(const qlin_weights* w, int64_t t, size_t*
 QLIN_API int qlin_gemv(const qlin_weights* w, const uint16_t* x_bf16, int64_t t, void* y, int y_dtype,
               const qlin_exec* ex);
 
-/* Workspace bytes qlin_gemm_a8 needs for T tokens against an N x K matrix. */
+/* Workspace bytes qlin_gemm_a8 should get for T tokens against an N x K
+ * matrix: the activation codes and scales (T*K + T*K/64*4 bytes, 256-byte
+ * aligned; the least a call with x_bf16 accepts) plus the weights expanded to
+ * int8 once per call (N*K bytes).  With the full size the GEMM reads int8
+ * weights through TMA (the faster kernel); with less, or none when the
+ * activations come pre-quantized, it expands the codes on chip. */
 QLIN_API int qlin_gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, size_t* bytes);
 
 /* Int8-route projection (prefill).  Weights must be Q3_G64, Q4_G64, Q5_G64 or Q6_G64
@@ -220,7 +225,9 @@ QLIN_API int qlin_gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, size_
  * S[t][n][g] = sum over the group of xq * q (int32, exact);
  * y[t][n] = sum_g (FP32(ws[n][g] * xs[t][g])) * S accumulated in FP32.
  * With flags & QLIN_DEBUG_GROUP_SUMS, S is also written to group_sums_dbg
- * int32[T][N][K/64].  The routing policy (T >= 129) is the caller's.
+ * int32[T][N][K/64].  The routing policy (T >= 129) is the caller's.  The
+ * workspace (see qlin_gemm_a8_workspace_bytes) is read and written; it must
+ * hold the activation part when x_bf16 is given (QLIN_ERR_WORKSPACE otherwise).
  * Accuracy: |y - y_ref| <= 5e-6 * sum_k |q ws||qa as| per element before the
  * BF16 output rounding.  ["NInfer int8-prefill artifact for the RTX 4090",
  * "What changes".] */

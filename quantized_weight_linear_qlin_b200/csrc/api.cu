@@ -346,7 +346,9 @@ int qlin_gemm_a8(const qlin_weights* w, const uint16_t* x_bf16, const int8_t* xq
   Exec e;
   if ((rc = make_exec(ex, &e))) return rc;
   if (fused) {
-    size_t need = gemm_a8_workspace_bytes(t, w->n, w->k, e.num_sms);
+    // at least the activation codes; the recommended size also holds the
+    // weights expanded to int8 (the faster kernel)
+    size_t need = gemm_a8_act_workspace_bytes(t, w->k);
     if (need > e.workspace_bytes || !e.workspace) return QLIN_ERR_WORKSPACE;
   }
   return launch_gemm_a8(*w, x_bf16, xq, xs, t, y, y_dtype, flags, group_sums_dbg, e);

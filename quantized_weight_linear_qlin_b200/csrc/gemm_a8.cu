@@ -220,78 +220,83 @@ __device__ __forceinline__ uint2 nibble_bytes(uint32_t w) {
                     __byte_perm(lo, hi, 0x7531));  // elements 4..7
 }
 
-// One 64-group of row r as 64 signed int8 codes q = u - 2^(BITS-1) in element
-// order (16 words).  `raw` is the stage's code plane (128-byte swizzled
-// nibbles, or for Q3 unswizzled 64-byte crumb rows), `hib` its second plane.
+// One 64-group as 64 signed int8 codes q = u - 2^(BITS-1) in element order
+// (16 words), from its code-plane words `cw` (Q3: 4 crumb words; else 8 nibble
+// words) and second-plane words `hw` (Q3 / Q5: 2 bit words; Q6: 4 crumb words).
 template <int BITS>
-__device__ __forceinline__ void expand_group(const uint8_t* raw, const uint8_t* hib, int r, int gi,
-                                             uint32_t* o) {
+__device__ __forceinline__ void expand_group_words(const uint32_t* cw, const uint32_t* hw, uint32_t* o) {
   // u + (128 - 2^(BITS-1)) then flip bit 7: the two's complement byte of q
   constexpr uint32_t ADD = BITS == 3 ? 0x7C7C7C7Cu : BITS == 4 ? 0x78787878u : BITS == 5 ? 0x70707070u
                                                                              : 0x60606060u;
   if constexpr (BITS == 3) {
-    const uint4 c = *(const uint4*)(raw + r * 64 + gi * 16);  // 4 crumb words: elements 16cw + 2s + o
-    const uint2 hh = *(const uint2*)(hib + r * 32 + gi * 8);  // bit words: elements 0..31, 32..63
-    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int cw = 0; cw < 4; ++cw) {
-      const uint32_t m0 = w[cw] & 0x03030303u;         // elements 0, 8, 1, 9
-      const uint32_t m1 = (w[cw] >> 2) & 0x03030303u;  // 2, 10, 3, 11
-      const uint32_t m2 = (w[cw] >> 4) & 0x03030303u;  // 4, 12, 5, 13
-      const uint32_t m3 = (w[cw] >> 6) & 0x03030303u;  // 6, 14, 7, 15
+    for (int c = 0; c < 4; ++c) {  // crumb word c: elements 16c + 2s + o
+      const uint32_t m0 = cw[c] & 0x03030303u;         // elements 0, 8, 1, 9
+      const uint32_t m1 = (cw[c] >> 2) & 0x03030303u;  // 2, 10, 3, 11
+      const uint32_t m2 = (cw[c] >> 4) & 0x03030303u;  // 4, 12, 5, 13
+      const uint32_t m3 = (cw[c] >> 6) & 0x03030303u;  // 6, 14, 7, 15
       const uint32_t e[4] = {__byte_perm(m0, m1, 0x6420), __byte_perm(m2, m3, 0x6420),
                              __byte_perm(m0, m1, 0x7531), __byte_perm(m2, m3, 0x7531)};
       // bit of element 2s+o of this crumb word: bit 16o + s of Hc
-      const uint32_t Hc = (cw < 2 ? hh.x : hh.y) >> (8 * (cw & 1));
+      const uint32_t Hc = hw[c >> 1] >> (8 * (c & 1));
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const uint32_t Hq = Hc >> (2 * q);  // elements 4q, 4q+1, 4q+2, 4q+3 at bits 0, 16, 1, 17
         const uint32_t b = ((Hq << 2) & 0x4u) | ((Hq >> 6) & 0x400u) | ((Hq << 17) & 0x40000u) |
                            ((Hq << 9) & 0x4000000u);
-        o[4 * cw + q] = ((e[q] | b) + ADD) ^ 0x80808080u;
+        o[4 * c + q] = ((e[q] | b) + ADD) ^ 0x80808080u;
       }
     }
   } else {
-    uint32_t h[4] = {0u, 0u, 0u, 0u};
-    if constexpr (BITS == 5) {
-      const uint2 hh = *(const uint2*)(hib + r * 32 + gi * 8);
-      h[0] = hh.x;
-      h[1] = hh.y;
-    } else if constexpr (BITS == 6) {
-      const uint4 hh = *(const uint4*)(hib + r * 64 + gi * 16);  // crumb words of elements 16c..
-      h[0] = hh.x;
-      h[1] = hh.y;
-      h[2] = hh.z;
-      h[3] = hh.w;
-    }
 #pragma unroll
-    for (int uu = 0; uu < 2; ++uu) {  // 16-byte units 2gi, 2gi+1 of the row = 64 elements
-      const uint4 c = *(const uint4*)(raw + sw128_offset(r, 2 * gi + uu));
-      const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int jw = 4 * uu + j;  // nibble word of the group: elements 8jw..8jw+7
-        uint2 e = nibble_bytes(wv[j]);
-        if constexpr (BITS == 5) {
-          // bit of element 8jw+2s+o at 16o + 4(jw&3) + s of word jw/4 -> bit 4 of its byte
-          const uint32_t hw = h[uu] >> (4 * j);
-          e.x |= ((hw << 4) & 0x10u) | ((hw >> 4) & 0x1000u) | ((hw << 19) & 0x100000u) |
-                 ((hw << 11) & 0x10000000u);
-          e.y |= ((hw << 2) & 0x10u) | ((hw >> 6) & 0x1000u) | ((hw << 17) & 0x100000u) |
-                 ((hw << 9) & 0x10000000u);
-        } else if constexpr (BITS == 6) {
-          // crumb of element 8jw+2s+o at 16o + 8(jw&1) + 2s of word jw/2 -> bits 4..5 of its byte
-          const uint32_t cj = h[jw >> 1] >> (8 * (jw & 1));
-          e.x |= ((cj << 4) & 0x30u) | ((cj >> 4) & 0x3000u) | ((cj << 18) & 0x300000u) |
-                 ((cj << 10) & 0x30000000u);
-          e.y |= (cj & 0x30u) | ((cj >> 8) & 0x3000u) | ((cj << 14) & 0x300000u) |
-                 ((cj << 6) & 0x30000000u);
-        }
-        o[8 * uu + 2 * j] = (e.x + ADD) ^ 0x80808080u;
-        o[8 * uu + 2 * j + 1] = (e.y + ADD) ^ 0x80808080u;
+    for (int jw = 0; jw < 8; ++jw) {  // nibble word jw: elements 8jw .. 8jw+7
+      uint2 e = nibble_bytes(cw[jw]);
+      if constexpr (BITS == 5) {
+        // bit of element 8jw+2s+o at 16o + 4(jw&3) + s of word jw/4 -> bit 4 of its byte
+        const uint32_t h = hw[jw >> 2] >> (4 * (jw & 3));
+        e.x |= ((h << 4) & 0x10u) | ((h >> 4) & 0x1000u) | ((h << 19) & 0x100000u) |
+               ((h << 11) & 0x10000000u);
+        e.y |= ((h << 2) & 0x10u) | ((h >> 6) & 0x1000u) | ((h << 17) & 0x100000u) |
+               ((h << 9) & 0x10000000u);
+      } else if constexpr (BITS == 6) {
+        // crumb of element 8jw+2s+o at 16o + 8(jw&1) + 2s of word jw/2 -> bits 4..5 of its byte
+        const uint32_t cj = hw[jw >> 1] >> (8 * (jw & 1));
+        e.x |= ((cj << 4) & 0x30u) | ((cj >> 4) & 0x3000u) | ((cj << 18) & 0x300000u) |
+               ((cj << 10) & 0x30000000u);
+        e.y |= (cj & 0x30u) | ((cj >> 8) & 0x3000u) | ((cj << 14) & 0x300000u) |
+               ((cj << 6) & 0x30000000u);
       }
+      o[2 * jw] = (e.x + ADD) ^ 0x80808080u;
+      o[2 * jw + 1] = (e.y + ADD) ^ 0x80808080u;
     }
   }
+}
+
+// The same for group gi of row r of a stage: `raw` is the stage's code plane
+// (128-byte swizzled nibbles, or for Q3 unswizzled 64-byte crumb rows), `hib`
+// its second plane.
+template <int BITS>
+__device__ __forceinline__ void expand_group(const uint8_t* raw, const uint8_t* hib, int r, int gi,
+                                             uint32_t* o) {
+  uint32_t cw[8], hw[4] = {0u, 0u, 0u, 0u};
+  if constexpr (BITS == 3) {
+    const uint4 c = *(const uint4*)(raw + r * 64 + gi * 16);
+    cw[0] = c.x; cw[1] = c.y; cw[2] = c.z; cw[3] = c.w;
+  } else {
+#pragma unroll
+    for (int uu = 0; uu < 2; ++uu) {  // 16-byte units 2gi, 2gi+1 of the row
+      const uint4 c = *(const uint4*)(raw + sw128_offset(r, 2 * gi + uu));
+      cw[4 * uu] = c.x; cw[4 * uu + 1] = c.y; cw[4 * uu + 2] = c.z; cw[4 * uu + 3] = c.w;
+    }
+  }
+  if constexpr (BITS == 3 || BITS == 5) {
+    const uint2 hh = *(const uint2*)(hib + r * 32 + gi * 8);
+    hw[0] = hh.x; hw[1] = hh.y;
+  } else if constexpr (BITS == 6) {
+    const uint4 hh = *(const uint4*)(hib + r * 64 + gi * 16);
+    hw[0] = hh.x; hw[1] = hh.y; hw[2] = hh.z; hw[3] = hh.w;
+  }
+  expand_group_words<BITS>(cw, hw, o);
 }
 
 template <int BITS, bool DEBUG>
@@ -609,15 +614,315 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Int8 group-sum GEMM on int8 weights expanded once per call.
+//   expand_i8_kernel  packed Q3..Q6 codes -> int8 [N][K] in the workspace
+//                     (one thread per (row, 64-group), bandwidth-bound);
+//   gemm_i8x_kernel   persistent CTAs over 128-row x 128-token tiles, row-tile
+//                     major (consecutive CTAs share a weight tile, which L2
+//                     then serves):
+//     warp 0     TMA: per stage a 128 x 128 B box of int8 weights and one of
+//                int8 activation codes (two 64-groups, 128-byte swizzle); its
+//                lanes cp.async the stage's weight and activation scales;
+//     warp 1     one elected thread issues tcgen05.mma.kind::i8 from both
+//                shared-memory operands (M = N = 128, K = 32), two per group,
+//                the first overwriting its accumulator, into one of three
+//                group-sum slots in tensor memory, and commits per group;
+//     warps 4-19 sixteen epilogue warps (row = lane of the warp's lane
+//                quarter, 32 tokens each, four warps per scheduler): read a
+//                group's sums with one tcgen05.ld, release the slot, and fold
+//                y += FP32(ws * as) * S in registers with paired FP32 multiplies
+//                and FMAs (S converts to FP32 exactly: |S| < 2^22); y is
+//                written once per tile.
+// No code expansion, no A operand written by the CUDA cores, and no output
+// tile in tensor memory: the tensor memory traffic per group is one read of
+// the sums.
+// ---------------------------------------------------------------------------
+constexpr int X_BK = 128;                   // K columns per stage: two 64-groups
+constexpr int X_NDS = 3;                    // group-sum slots
+constexpr int X_NEPI = 16;                  // epilogue warps: 4 lane quarters x 4 token blocks
+constexpr int X_WEPI0 = 4;
+constexpr int X_THREADS = (X_WEPI0 + X_NEPI) * 32;  // warps 0..3 control, 4..19 epilogue
+
+struct __align__(1024) XStage {
+  uint8_t a[BM * 128];      // int8 weights, 128 rows x 128 columns (swizzled)
+  uint8_t b[BN * 128];      // int8 activations, 128 tokens x 128 columns (swizzled)
+  float xsb[2 * BN];        // activation scales [group][token]
+  __half wsb[BM * 2];       // weight scales [row][group]
+};
+constexpr int X_NS = 6;
+struct XSmem {
+  XStage st[X_NS];
+  uint64_t full[X_NS], empty[X_NS];
+  uint64_t sfull[X_NDS], sfree[X_NDS];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int BITS>
+__global__ void expand_i8_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ hib,
+                                 int64_t n, int64_t k, int8_t* __restrict__ out) {
+  const int64_t ng = k / 64;
+  for (int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; item < n * ng;
+       item += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = item / ng, g = item - r * ng;
+    uint32_t cw[8], hw[4] = {0u, 0u, 0u, 0u};
+    if constexpr (BITS == 3) {
+      const uint4 c = __ldcs((const uint4*)(codes + r * (k / 4) + g * 16));
+      cw[0] = c.x; cw[1] = c.y; cw[2] = c.z; cw[3] = c.w;
+    } else {
+      const uint4* src = (const uint4*)(codes + r * (k / 2) + g * 32);
+      const uint4 c0 = __ldcs(src), c1 = __ldcs(src + 1);
+      cw[0] = c0.x; cw[1] = c0.y; cw[2] = c0.z; cw[3] = c0.w;
+      cw[4] = c1.x; cw[5] = c1.y; cw[6] = c1.z; cw[7] = c1.w;
+    }
+    if constexpr (BITS == 3 || BITS == 5) {
+      const uint2 hh = __ldcs((const uint2*)(hib + r * (k / 8) + g * 8));
+      hw[0] = hh.x; hw[1] = hh.y;
+    } else if constexpr (BITS == 6) {
+      const uint4 hh = __ldcs((const uint4*)(hib + r * (k / 4) + g * 16));
+      hw[0] = hh.x; hw[1] = hh.y; hw[2] = hh.z; hw[3] = hh.w;
+    }
+    uint32_t o[16];
+    expand_group_words<BITS>(cw, hw, o);
+    uint4* dst = (uint4*)(out + r * k + g * 64);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+  }
+}
+
+template <bool DEBUG>
+__global__ void __launch_bounds__(X_THREADS, 1)
+    gemm_i8x_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_act,
+                    GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  XSmem& sm = *reinterpret_cast<XSmem*>((void*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ng = args.k / 64;
+  const int nchunks = (int)(args.k / X_BK);
+  const int64_t my_tiles = (args.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < X_NS; ++s) {
+      mbar_init(&sm.full[s], 1 + 32);  // TMA issue + 32 scale-copy arrivals
+      mbar_init(&sm.empty[s], 1 + X_NEPI);  // the MMA commit + the epilogue warps (scales read)
+    }
+    for (int d = 0; d < X_NDS; ++d) {
+      mbar_init(&sm.sfull[d], 1);
+      mbar_init(&sm.sfree[d], X_NEPI);
+    }
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_act);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // the activation codes and the expanded weights come from the kernels
+    // launched just before
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    int issued = 0;
+    Ring ring{0, 0};
+    bool ok = true;
+    for (int64_t it = 0; it < my_tiles && ok; ++it) {
+      const int64_t tile = blockIdx.x + it * gridDim.x;
+      const int64_t n0 = (tile / args.tiles_t) * BM, t0 = (tile % args.tiles_t) * BN;
+      for (int kc = 0; kc < nchunks; ++kc) {
+        const int s = ring.slot;
+        if (!__all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.empty[s], (uint32_t)(ring.phase ^ 1)))) {
+          if (lane == 0) set_abort(sm, args.dev_status);
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(BM * 128 + BN * 128));
+          tma_load_2d(sm.st[s].a, &tm_w, &sm.full[s], kc * X_BK, (int)n0);
+          tma_load_2d(sm.st[s].b, &tm_act, &sm.full[s], kc * X_BK, (int)t0);
+        }
+        // weight scales: two groups (4 bytes) per row; activation scales [group][token]
+        for (int rr = lane; rr < BM; rr += 32) {
+          const int64_t grow = n0 + rr;
+          if (grow < args.n) cp_async_4(&sm.st[s].wsb[rr * 2], args.ws + grow * ng + (int64_t)kc * 2);
+        }
+        for (int tt = lane; tt < BN; tt += 32) {
+          const int64_t gt = t0 + tt;
+          if (gt < args.t)
+            for (int gi = 0; gi < 2; ++gi)
+              cp_async_4(&sm.st[s].xsb[gi * BN + tt], args.xs + gt * ng + (int64_t)kc * 2 + gi);
+        }
+        cp_async_arrive_noinc(&sm.full[s]);
+        ++issued;
+        ring.next(X_NS);
+      }
+    }
+    if (lane == 0) {
+      Ring r2{0, 0};
+      for (int i = 0; i < issued; ++i) {
+        if (i + X_NS >= issued) mbar_wait(&sm.full[r2.slot], (uint32_t)r2.phase);
+        r2.next(X_NS);
+      }
+    }
+  } else if (warp == 1) {
+    const uint32_t idesc = idesc_i8(BM, BN);
+    Ring ring{0, 0}, dr{0, 0};
+    bool ok = true;
+    for (int64_t it = 0; it < my_tiles && ok; ++it) {
+      for (int kc = 0; kc < nchunks && ok; ++kc) {
+        const int s = ring.slot;
+        ok = __all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.full[s], (uint32_t)ring.phase));
+        if (!ok) break;
+        const uint32_t as = smem_u32(sm.st[s].a), bs = smem_u32(sm.st[s].b);
+        for (int gi = 0; gi < 2 && ok; ++gi) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.sfree[dr.slot], (uint32_t)(dr.phase ^ 1)) && !aborted(sm));
+          if (!ok) break;
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)  // K = 32 int8 = 32 bytes of the swizzled rows
+              mma_i8_ss(tmem + dr.slot * BN, sdesc_k_sw128(as + gi * 64 + kk * 32),
+                        sdesc_k_sw128(bs + gi * 64 + kk * 32), idesc, kk ? 1u : 0u);
+            tc_commit(&sm.sfull[dr.slot]);
+          }
+          __syncwarp();
+          dr.next(X_NDS);
+        }
+        if (!ok) break;
+        if (elect_one()) tc_commit(&sm.empty[s]);  // the stage's operands are read once these finish
+        __syncwarp();
+        ring.next(X_NS);
+      }
+    }
+    if (!ok && lane == 0) set_abort(sm, args.dev_status);
+  } else if (warp >= X_WEPI0) {
+    // warp w reads tensor-memory lanes 32 * (w % 4) .. +31 (its rows) and the
+    // 32 tokens of its column block
+    const int quarter = warp & 3, cblk = (warp - X_WEPI0) >> 2;
+    const int row = quarter * 32 + lane;
+    const int col0 = cblk * 32;
+    const uint32_t lane_ofs = (uint32_t)(quarter * 32) << 16;
+    Ring ring{0, 0}, dr{0, 0};
+    bool ok = true;
+    for (int64_t it = 0; it < my_tiles && ok; ++it) {
+      const int64_t tile = blockIdx.x + it * gridDim.x;
+      const int64_t n0 = (tile / args.tiles_t) * BM, t0 = (tile % args.tiles_t) * BN;
+      const int64_t grow = n0 + row;
+      float2 y2[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) y2[j] = make_float2(0.0f, 0.0f);
+      for (int kc = 0; kc < nchunks && ok; ++kc) {
+        const int s = ring.slot;
+        // the stage's scales have landed once its barrier completed (acquire)
+        ok = __all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.full[s], (uint32_t)ring.phase));
+        if (!ok) break;
+        const uint32_t wsw = *(const uint32_t*)&sm.st[s].wsb[row * 2];
+        for (int gi = 0; gi < 2 && ok; ++gi) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.sfull[dr.slot], (uint32_t)dr.phase));
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t sv[32];
+          tmem_ld_x32(tmem + lane_ofs + dr.slot * BN + col0, sv);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.sfree[dr.slot]);  // the slot may be overwritten now
+          if (DEBUG && grow < args.n) {
+            int32_t* dp = args.sums_dbg + ((t0 + col0) * args.n + grow) * ng + (int64_t)kc * 2 + gi;
+            const int64_t dstep = args.n * ng;
+#pragma unroll 4
+            for (int j = 0; j < 32; ++j, dp += dstep)
+              if (t0 + col0 + j < args.t) *dp = (int32_t)sv[j];
+          }
+          const float wsc = __half2float(__ushort_as_half((unsigned short)(wsw >> (16 * gi))));
+          const float2 w2 = make_float2(wsc, wsc);
+          const float4* xsg = (const float4*)(sm.st[s].xsb + gi * BN + col0);
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 xv = xsg[j4];
+            // |S| < 2^22: the int32 sum converts to FP32 exactly
+            const float2 f0 = make_float2(__int2float_rn((int)sv[4 * j4]), __int2float_rn((int)sv[4 * j4 + 1]));
+            const float2 f1 =
+                make_float2(__int2float_rn((int)sv[4 * j4 + 2]), __int2float_rn((int)sv[4 * j4 + 3]));
+            y2[2 * j4] = __ffma2_rn(__fmul2_rn(w2, make_float2(xv.x, xv.y)), f0, y2[2 * j4]);
+            y2[2 * j4 + 1] = __ffma2_rn(__fmul2_rn(w2, make_float2(xv.z, xv.w)), f1, y2[2 * j4 + 1]);
+          }
+          dr.next(X_NDS);
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[s]);  // the stage's scales are consumed
+        ring.next(X_NS);
+      }
+      if (!ok) {
+        set_abort(sm, args.dev_status);
+        break;
+      }
+      if (grow < args.n) {
+        const int jmax = (int)min((int64_t)32, args.t - (t0 + col0));
+        const int64_t base = (t0 + col0) * args.n + grow;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j < jmax) {
+            const float v = (j & 1) ? y2[j >> 1].y : y2[j >> 1].x;
+            if (args.y_dtype == QLIN_OUT_F32)
+              ((float*)args.y)[base + (int64_t)j * args.n] = v;
+            else
+              ((__nv_bfloat16*)args.y)[base + (int64_t)j * args.n] = __float2bfloat16_rn(v);
+          }
+        }
+      }
+    }
+  }
+
+  // Every group sum's completion was observed by the epilogue before this
+  // point -- unless a wait timed out; then give the tensor core ample time
+  // (1 ms) before the tensor memory is released.
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (aborted(sm)) {
+      const unsigned long long t0 = global_ns();
+      while (global_ns() - t0 < 1000000ull) {
+      }
+    }
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
-size_t gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, int num_sms) {
-  (void)n;
-  (void)num_sms;
-  size_t xq = ((size_t)t * k + 255) / 256 * 256;
-  size_t xs = (size_t)t * (k / 64) * sizeof(float);
-  return xq + xs;
+// Workspace: xq int8 [T][K] | xs FP32 [T][K/64] | the weights expanded to int8
+// [N][K] (each part 256-byte aligned).  A workspace too small for the last
+// part runs the kernel that expands the codes in tensor memory instead.
+struct A8Ws {
+  size_t xq, xs, w8, total, act_total;
+};
+static A8Ws a8_ws(int64_t t, int64_t n, int64_t k) {
+  A8Ws L;
+  L.xq = 0;
+  L.xs = ((size_t)t * k + 255) / 256 * 256;
+  L.act_total = L.xs + (size_t)t * (k / 64) * sizeof(float);
+  L.w8 = (L.act_total + 255) / 256 * 256;
+  L.total = L.w8 + (size_t)n * k;
+  return L;
 }
+
+size_t gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, int num_sms) {
+  (void)num_sms;
+  return a8_ws(t, n, k).total;
+}
+size_t gemm_a8_act_workspace_bytes(int64_t t, int64_t k) { return a8_ws(t, 0, k).act_total; }
 
 int launch_quantize_act(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* xs,
                         const Exec& ex) {
@@ -650,20 +955,81 @@ static int launch_a8(const CUtensorMap& tm_codes, const CUtensorMap& tm_hib, con
   return cuda_status(cudaLaunchKernelEx(&cfg, gemm_a8_kernel<BITS, DEBUG>, tm_codes, tm_hib, tm_act, args));
 }
 
+template <bool DEBUG>
+static int launch_i8x(const CUtensorMap& tm_w, const CUtensorMap& tm_act, const GemmArgs& args, int grid,
+                      const Exec& ex) {
+  const size_t smem = sizeof(XSmem) + 1024;
+  const cudaError_t e0 = set_smem_once<gemm_i8x_kernel<DEBUG>>((int)smem);
+  if (e0 != cudaSuccess) return cuda_status(e0);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(X_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = ex.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, gemm_i8x_kernel<DEBUG>, tm_w, tm_act, args));
+}
+
 int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, const float* xs,
                    int64_t t, void* y, int y_dtype, uint32_t flags, int32_t* sums_dbg,
                    const Exec& ex) {
   const int64_t n = w.n, k = w.k;
+  const A8Ws wl = a8_ws(t, n, k);
+  const bool expanded = ex.workspace != nullptr && ex.workspace_bytes >= wl.total;
+  const int bits = w.fmt == QLIN_Q3_G64 ? 3 : w.fmt == QLIN_Q4_G64 ? 4 : w.fmt == QLIN_Q5_G64 ? 5 : 6;
+  int8_t* w8 = expanded ? (int8_t*)((uint8_t*)ex.workspace + wl.w8) : nullptr;
+  if (expanded) {
+    // the codes as int8 [N][K], once per call (bandwidth-bound)
+    const int64_t items = n * (k / 64);
+    const int64_t blocks = std::min<int64_t>((items + 255) / 256, (int64_t)ex.num_sms * 16);
+    const uint8_t* c = (const uint8_t*)w.codes;
+    const uint8_t* h = (const uint8_t*)w.hibits;
+    switch (bits) {
+      case 3: expand_i8_kernel<3><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8); break;
+      case 4: expand_i8_kernel<4><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8); break;
+      case 5: expand_i8_kernel<5><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8); break;
+      default: expand_i8_kernel<6><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8); break;
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   if (x != nullptr) {
     // quantize into the workspace first
     int8_t* wq = (int8_t*)ex.workspace;
-    float* wsc = (float*)((uint8_t*)ex.workspace + ((size_t)t * k + 255) / 256 * 256);
+    float* wsc = (float*)((uint8_t*)ex.workspace + wl.xs);
     int rc = launch_quantize_act(x, t, k, wq, wsc, ex);
     if (rc != QLIN_OK) return rc;
     xq = wq;
     xs = wsc;
   }
-  const int bits = w.fmt == QLIN_Q3_G64 ? 3 : w.fmt == QLIN_Q4_G64 ? 4 : w.fmt == QLIN_Q5_G64 ? 5 : 6;
+  if (expanded) {
+    CUtensorMap tm_w, tm_act;
+    int rc = encode_tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w8, (uint64_t)k, (uint64_t)n, (uint64_t)k,
+                            128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    rc = encode_tmap_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)k, (uint64_t)t, (uint64_t)k,
+                        128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    GemmArgs args;
+    args.ws = (const __half*)w.scales;
+    args.xs = xs;
+    args.y = y;
+    args.sums_dbg = sums_dbg;
+    args.dev_status = ex.dev_status;
+    args.n = n;
+    args.k = k;
+    args.t = t;
+    args.tiles_t = (t + BN - 1) / BN;
+    args.tiles = args.tiles_t * ((n + BM - 1) / BM);
+    args.y_dtype = y_dtype;
+    const int grid = (int)std::min<int64_t>(args.tiles, ex.num_sms);
+    return (flags & QLIN_DEBUG_GROUP_SUMS) ? launch_i8x<true>(tm_w, tm_act, args, grid, ex)
+                                           : launch_i8x<false>(tm_w, tm_act, args, grid, ex);
+  }
   // code plane: 128-byte swizzled nibble rows, or (Q3) unswizzled 64-byte crumb rows per stage
   const uint64_t crow = (uint64_t)(bits == 3 ? k / 4 : k / 2);
   CUtensorMap tm_codes, tm_hib, tm_act;

@@ -38,6 +38,7 @@ size_t gemv_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms);
 int launch_gemv(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                 const Exec& ex);
 size_t gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, int num_sms);
+size_t gemm_a8_act_workspace_bytes(int64_t t, int64_t k);
 int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, const float* xs,
                    int64_t t, void* y, int y_dtype, uint32_t flags, int32_t* sums_dbg,
                    const Exec& ex);

@@ -364,7 +364,14 @@ def test_gemv_several_units_per_cta(fmt, t):
 # ---------------------------------------------------------------------------
 # int8 route
 # ---------------------------------------------------------------------------
-def run_gemm_a8(pw, x, fused=True, debug=True, y_dtype=q.OUT_F32):
+def act_ws_bytes(t, k):
+    """The activation part of the int8 route's workspace (codes + scales)."""
+    return (t * k + 255) // 256 * 256 + t * (k // 64) * 4
+
+
+def run_gemm_a8(pw, x, fused=True, debug=True, y_dtype=q.OUT_F32, full_ws=True):
+    """full_ws: the recommended workspace (weights expanded to int8 once, TMA-fed
+    GEMM); else only the activation part (codes expanded on chip)."""
     t, k = x.shape
     n = pw.n
     xd = x.to(DEV)
@@ -373,7 +380,7 @@ def run_gemm_a8(pw, x, fused=True, debug=True, y_dtype=q.OUT_F32):
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     flags = q.DEBUG_GROUP_SUMS if debug else 0
     if fused:
-        ws = q.Workspace(DEV).ensure(q.qlin_gemm_a8_workspace_bytes(t, n, k))
+        ws = q.Workspace(DEV).ensure(q.qlin_gemm_a8_workspace_bytes(t, n, k) if full_ws else act_ws_bytes(t, k))
         q.qlin_gemm_a8(pw, y, x=xd, y_dtype=y_dtype, flags=flags, sums_dbg=dbg, workspace=ws,
                        dev_status=status)
     else:
@@ -387,15 +394,16 @@ def run_gemm_a8(pw, x, fused=True, debug=True, y_dtype=q.OUT_F32):
     return y, dbg
 
 
+@pytest.mark.parametrize("full_ws", [True, False])
 @pytest.mark.parametrize("fmt", ["q4", "q5", "q3", "q6"])
 @pytest.mark.parametrize("n,k,t", [(128, 256, 128), (256, 512, 130), (200, 640, 257), (384, 1152, 1),
                                    (128, 5120, 64)])
-def test_gemm_a8_group_sums_bit_exact_and_output(fmt, n, k, t):
+def test_gemm_a8_group_sums_bit_exact_and_output(fmt, n, k, t, full_ws):
     w = synth.weights_f32(n, k, seed=400 + n + k)
     x = synth.activations_bf16(t, k, seed=500 + t)
     ref = oracle.pack(FMTS[fmt], w.numpy())
     pw = pack_gpu(FMTS[fmt], w.to(DEV), allow_a8=True)
-    y, dbg = run_gemm_a8(pw, x, fused=True, debug=True)
+    y, dbg = run_gemm_a8(pw, x, fused=True, debug=True, full_ws=full_ws)
     qa, as_ = oracle.quantize_act(bits16(x))
     S = oracle.group_sums(ref, qa)
     assert np.array_equal(dbg.cpu().numpy(), S)
