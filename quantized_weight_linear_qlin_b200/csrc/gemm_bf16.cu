@@ -9,16 +9,21 @@
 // while W (96 x 5120, 1 MB) stays in L2.  So the tokens go on M (128 per tile)
 // and the weight rows on N (N padded to a multiple of 16, at most 256); a CTA
 // takes one or two 128-token sub-tiles, and the K range of a tile is split
-// over several CTAs so that all of them run in one wave:
+// over the CTAs of one thread-block cluster (up to 16) so that all of them run
+// in one wave:
 //   warp 0     TMA: per stage a 64-column box of 128 token rows of x for each
 //              sub-tile and one of the N weight rows (128-byte swizzle);
 //   warp 1     one elected thread issues tcgen05.mma.kind::f16 (BF16 x BF16 ->
 //              FP32, M = 128, N = NP, K = 16), four per stage and sub-tile,
 //              one tensor-memory accumulator per sub-tile;
 //   warps 4-7  the epilogue reads the accumulator with tcgen05.ld (thread =
-//              token) and writes y, or, when K is split, an FP32 partial that
-//              gemm_bf16_reduce sums over the parts in a fixed order.
+//              token) and writes y, or, when K is split, the CTA's FP32
+//              partial into its own shared memory; after a cluster barrier
+//              every CTA of the cluster sums a share of the tile's outputs over
+//              the parts' shared memories (distributed shared memory) in part
+//              order and writes y.  No partial leaves the chip.
 #include <algorithm>
+#include <atomic>
 
 #include "qlin_internal.cuh"
 
@@ -47,15 +52,43 @@ struct B16Cfg {
   static_assert(COLS <= 512, "tensor memory");
   static_assert(A_SUB % 1024 == 0 && STAGE % 1024 == 0, "1024-byte aligned operands");
   static_assert(NS >= 2, "pipeline needs two stages");
+  static_assert((size_t)MT * B16_BM * (NP + 4) * 4 <= (size_t)NS * STAGE, "partial fits the stage buffers");
 };
 
 struct B16Args {
-  void* out;          // y [T][N] (parts == 1) or FP32 partials [parts][T][N]
+  void* out;          // y [T][N]
   int32_t* dev_status;
   int64_t n, k, t;
-  int tiles, parts;   // token tiles, K parts per tile
-  int out_dtype;      // QLIN_OUT_BF16 / QLIN_OUT_F32 (parts == 1), F32 for partials
+  int tiles, parts;   // token tiles, K parts per tile (= the cluster size)
+  int out_dtype;      // QLIN_OUT_BF16 / QLIN_OUT_F32
 };
+
+// The FP32 partial of a CTA in its shared memory: [MT * 128 tokens][NP + 4]
+// (the 4-float pad keeps the 16-byte row writes of a warp on distinct banks).
+template <int NP>
+constexpr int red_stride() { return NP + 4; }
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
 
 template <int NP, int MT>
 __global__ void __launch_bounds__(B16_THREADS, 1)
@@ -159,12 +192,14 @@ __global__ void __launch_bounds__(B16_THREADS, 1)
     if (!__any_sync(0xffffffffu, *abort_flag != 0) && __all_sync(0xffffffffu, mbar_wait(acc_full, 0))) {
       tc_fence_after();
       const uint32_t lane_ofs = (uint32_t)(quarter * 32) << 16;
-      const bool f32 = args.parts > 1 || args.out_dtype == QLIN_OUT_F32;
+      const bool f32 = args.out_dtype == QLIN_OUT_F32;
       const bool vec = (args.n & 3) == 0;  // rows of y start on 16 bytes (FP32) / 8 bytes (BF16)
+      float* red = (float*)base;           // the stage buffers are idle once the accumulator is complete
 #pragma unroll 1
       for (int m = 0; m < MT; ++m) {
-        const int64_t tok = ((int64_t)tile * MT + m) * B16_BM + quarter * 32 + lane;
-        const int64_t obase = ((int64_t)part * args.t + tok) * args.n;
+        const int ltok = m * B16_BM + quarter * 32 + lane;
+        const int64_t tok = (int64_t)tile * MT * B16_BM + ltok;
+        const int64_t obase = tok * args.n;
 #pragma unroll 1
         for (int c0 = 0; c0 < NP; c0 += 16) {
           if (c0 >= args.n) break;
@@ -173,6 +208,14 @@ __global__ void __launch_bounds__(B16_THREADS, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) asm volatile("" : "+r"(v[j]));
+          if (args.parts > 1) {
+            float4* o = (float4*)(red + ltok * red_stride<NP>() + c0);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              o[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                  __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+            continue;
+          }
           if (tok >= args.t) continue;
           if (vec && c0 + 16 <= args.n) {
             if (f32) {
@@ -208,6 +251,57 @@ __global__ void __launch_bounds__(B16_THREADS, 1)
     }
   }
 
+  if (args.parts > 1) {
+    // Every CTA of the cluster reaches both barriers, on every path (a timed
+    // out CTA contributes whatever its partial holds; its status is set).
+    __syncthreads();
+    cluster_sync_all();
+    // rank r sums outputs [r * E / P, (r + 1) * E / P) of the tile, E = its
+    // tokens x NP / 4 four-column groups, over the P partials in part order
+    constexpr int C4 = NP / 4;
+    constexpr int E = MT * B16_BM * C4;
+    const int P = args.parts;
+    const uint32_t r = cluster_rank();
+    const int lo = (int)((int64_t)r * E / P), hi = (int)((int64_t)(r + 1) * E / P);
+    const uint32_t red_s = smem_u32(base);
+    const bool f32 = args.out_dtype == QLIN_OUT_F32;
+    const bool vec = (args.n & 3) == 0;
+    for (int idx = lo + (int)threadIdx.x; idx < hi; idx += B16_THREADS) {
+      const int ltok = idx / C4, col = (idx - ltok * C4) * 4;
+      const int64_t tok = (int64_t)tile * MT * B16_BM + ltok;
+      if (tok >= args.t || col >= args.n) continue;
+      const uint32_t off = (uint32_t)(ltok * red_stride<NP>() + col) * 4u;
+      float4 acc = ld_dsmem_v4(map_to_rank(red_s + off, 0));
+      for (int p = 1; p < P; ++p) {
+        const float4 v = ld_dsmem_v4(map_to_rank(red_s + off, (uint32_t)p));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      const int64_t o = tok * args.n + col;
+      if (vec) {
+        if (f32) {
+          *(float4*)((float*)args.out + o) = acc;
+        } else {
+          const __nv_bfloat162 a01 = __floats2bfloat162_rn(acc.x, acc.y);
+          const __nv_bfloat162 a23 = __floats2bfloat162_rn(acc.z, acc.w);
+          *(uint2*)((__nv_bfloat16*)args.out + o) = make_uint2(*(const uint32_t*)&a01, *(const uint32_t*)&a23);
+        }
+      } else {
+        const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+        for (int j = 0; j < 4 && col + j < args.n; ++j) {
+          if (f32)
+            ((float*)args.out)[o + j] = a[j];
+          else
+            ((__nv_bfloat16*)args.out)[o + j] = __float2bfloat16_rn(a[j]);
+        }
+      }
+    }
+    // no CTA leaves (and frees its shared memory) while another still reads it
+    cluster_sync_all();
+  }
+
   // The accumulator's completion was observed by the epilogue before this
   // point -- unless a wait timed out; then give the tensor core ample time
   // (1 ms) before the tensor memory is released.
@@ -224,51 +318,89 @@ __global__ void __launch_bounds__(B16_THREADS, 1)
   }
 }
 
-// y[i] = sum over the parts, in part order, of the FP32 partials.
-__global__ void gemm_bf16_reduce_kernel(const float* __restrict__ partials, int parts, int64_t count,
-                                        void* y, int y_dtype) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    float v = partials[i];
-    for (int p = 1; p < parts; ++p) v += partials[(int64_t)p * count + i];
-    if (y_dtype == QLIN_OUT_F32)
-      ((float*)y)[i] = v;
-    else
-      ((__nv_bfloat16*)y)[i] = __float2bfloat16_rn(v);
-  }
-}
-
 int np_of(int64_t n) { return n <= 64 ? 64 : n <= 96 ? 96 : n <= 128 ? 128 : 256; }
 // 128-token sub-tiles per CTA: two from 1024 tokens on (the weight box is then
-// read once per 256 tokens), one below (more CTAs for short prompts).
-int mt_of(int64_t t) { return t >= 1024 ? 2 : 1; }
+// read once per 256 tokens), one below (more CTAs for short prompts) and for
+// N = 256 (the partial of two sub-tiles would not fit the stage buffers).
+int mt_of(int64_t t, int np) { return t >= 1024 && np <= 128 ? 2 : 1; }
 
-// K parts per token tile: as many as keep all the work items in one wave of
-// CTAs, each part at least two 64-column stages.
-int parts_of(int64_t t, int64_t k, int num_sms) {
-  const int64_t tiles = (t + (int64_t)B16_BM * mt_of(t) - 1) / ((int64_t)B16_BM * mt_of(t));
+constexpr int kMaxParts = 16;  // non-portable cluster size; 8 where the device refuses 16
+
+// Clusters of `p` CTAs that can be resident at once on this device (cached per
+// device and configuration); 0 when the device refuses the cluster size.
+template <int NP, int MT>
+int max_clusters(int p) {
+  static std::atomic<int> cache[64][kMaxParts + 1];  // value + 1; 0 = not asked yet
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int c = cache[dev][p].load(std::memory_order_relaxed);
+  if (c > 0) return c - 1;
+  using C = B16Cfg<NP, MT>;
+  int n = 0;
+  if (set_smem_once<gemm_bf16_tok_kernel<NP, MT>>((int)C::SMEM) == cudaSuccess &&
+      (p <= 8 || cudaFuncSetAttribute(gemm_bf16_tok_kernel<NP, MT>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                      1) == cudaSuccess)) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p);
+    cfg.blockDim = dim3(B16_THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_tok_kernel<NP, MT>, &cfg) != cudaSuccess) n = 0;
+  }
+  (void)cudaGetLastError();  // a refused size is an answer, not an error of this call
+  cache[dev][p].store(n + 1, std::memory_order_relaxed);
+  return n;
+}
+
+// K parts per token tile (the cluster size): as many as keep every tile's
+// cluster resident in one wave, at most one per SM per tile and each part at
+// least two 64-column stages.
+template <int NP, int MT>
+int parts_for(int64_t tiles, int64_t k, int num_sms) {
   const int64_t nkb = k / B16_BK;
   int64_t p = std::max<int64_t>(1, num_sms / tiles);
-  p = std::min<int64_t>(p, std::max<int64_t>(1, nkb / 2));
+  p = std::min<int64_t>({p, std::max<int64_t>(1, nkb / 2), (int64_t)kMaxParts});
+  for (; p > 1; --p)
+    if (max_clusters<NP, MT>((int)p) >= tiles) break;
   return (int)p;
 }
 
 template <int NP, int MT>
-int launch_np(const CUtensorMap& mx, const CUtensorMap& mw, const B16Args& a, cudaStream_t st) {
+int launch_np(const CUtensorMap& mx, const CUtensorMap& mw, const B16Args& a, int num_sms, cudaStream_t st) {
   using C = B16Cfg<NP, MT>;
   const cudaError_t e0 = set_smem_once<gemm_bf16_tok_kernel<NP, MT>>((int)C::SMEM);
   if (e0 != cudaSuccess) return cuda_status(e0);
-  gemm_bf16_tok_kernel<NP, MT><<<(unsigned)(a.tiles * a.parts), B16_THREADS, C::SMEM, st>>>(mx, mw, a);
-  return cuda_status(cudaGetLastError());
+  B16Args args = a;
+  args.parts = parts_for<NP, MT>(a.tiles, a.k, num_sms);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(args.tiles * args.parts));
+  cfg.blockDim = dim3(B16_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)args.parts;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, gemm_bf16_tok_kernel<NP, MT>, mx, mw, args));
 }
 
 template <int MT>
-int launch_mt(int np, const CUtensorMap& mx, const CUtensorMap& mw, const B16Args& a, cudaStream_t st) {
+int launch_mt(int np, const CUtensorMap& mx, const CUtensorMap& mw, const B16Args& a, int num_sms,
+              cudaStream_t st) {
   switch (np) {
-    case 64: return launch_np<64, MT>(mx, mw, a, st);
-    case 96: return launch_np<96, MT>(mx, mw, a, st);
-    case 128: return launch_np<128, MT>(mx, mw, a, st);
-    default: return launch_np<256, MT>(mx, mw, a, st);
+    case 64: return launch_np<64, MT>(mx, mw, a, num_sms, st);
+    case 96: return launch_np<96, MT>(mx, mw, a, num_sms, st);
+    case 128: return launch_np<128, MT>(mx, mw, a, num_sms, st);
+    default: return launch_np<256, 1>(mx, mw, a, num_sms, st);
   }
 }
 
@@ -280,10 +412,7 @@ bool gemm_bf16_tok_supported(const qlin_weights& w, int64_t t) {
   return w.fmt == QLIN_BF16 && w.n <= 256 && w.k % B16_BK == 0 && t > 64 && t <= (int64_t)INT32_MAX / 2;
 }
 
-size_t gemm_bf16_tok_workspace_bytes(const qlin_weights& w, int64_t t, int num_sms) {
-  const int parts = parts_of(t, w.k, num_sms);
-  return parts > 1 ? (size_t)parts * t * w.n * sizeof(float) : 0;
-}
+size_t gemm_bf16_tok_workspace_bytes(const qlin_weights&, int64_t, int) { return 0; }
 
 int launch_gemm_bf16_tok(const qlin_weights& w, const uint16_t* x, int64_t t, void* y, int y_dtype,
                          const Exec& ex) {
@@ -296,22 +425,17 @@ int launch_gemm_bf16_tok(const qlin_weights& w, const uint16_t* x, int64_t t, vo
                       (uint64_t)w.k * 2, B16_BK, (uint32_t)np, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   B16Args a;
-  const int mt = mt_of(t);
-  a.parts = parts_of(t, w.k, ex.num_sms);
+  const int mt = mt_of(t, np);
   a.tiles = (int)((t + (int64_t)B16_BM * mt - 1) / ((int64_t)B16_BM * mt));
-  a.out = a.parts > 1 ? ex.workspace : y;
+  a.parts = 1;  // launch_np sets the cluster size
+  a.out = y;
   a.dev_status = ex.dev_status;
   a.n = w.n;
   a.k = w.k;
   a.t = t;
   a.out_dtype = y_dtype;
-  rc = mt == 2 ? launch_mt<2>(np, mx, mw, a, ex.stream) : launch_mt<1>(np, mx, mw, a, ex.stream);
-  if (rc != QLIN_OK || a.parts == 1) return rc;
-  const int64_t count = t * w.n;
-  const int64_t blocks = std::min<int64_t>((count + 255) / 256, (int64_t)ex.num_sms * 8);
-  gemm_bf16_reduce_kernel<<<(unsigned)blocks, 256, 0, ex.stream>>>((const float*)ex.workspace, a.parts,
-                                                                  count, y, y_dtype);
-  return cuda_status(cudaGetLastError());
+  return mt == 2 ? launch_mt<2>(np, mx, mw, a, ex.num_sms, ex.stream)
+                 : launch_mt<1>(np, mx, mw, a, ex.num_sms, ex.stream);
 }
 
 }  // namespace qlin

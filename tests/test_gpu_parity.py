@@ -256,12 +256,14 @@ def test_gemv_bf16_weights_prefill_sizes(t):
 
 @pytest.mark.parametrize("n,k,t,y_dtype", [(80, 1024, 300, q.OUT_BF16), (256, 640, 129, q.OUT_F32),
                                            (16, 4096, 2000, q.OUT_F32), (200, 192, 777, q.OUT_BF16),
-                                           (96, 5120, 1100, q.OUT_BF16), (64, 2048, 1025, q.OUT_F32)])
+                                           (96, 5120, 1100, q.OUT_BF16), (64, 2048, 1025, q.OUT_F32),
+                                           (90, 512, 333, q.OUT_BF16), (250, 1024, 1500, q.OUT_F32)])
 def test_gemv_bf16_weights_prefill_ragged_n(n, k, t, y_dtype):
     """Small BF16 projections at prefill sizes: N padded inside the kernel
-    (80 -> 96, 200 -> 256), few K stages (K = 192: one part), BF16 and FP32 out;
-    1100 and 1025 tokens leave the last CTA's second 128-token sub-tile wholly
-    or all but one token out of range."""
+    (80 -> 96, 200 and 250 -> 256), few K stages (K = 192: one part), BF16 and
+    FP32 out; 1100 and 1025 tokens leave the last CTA's second 128-token
+    sub-tile wholly or all but one token out of range; N = 90 and 250 are not
+    multiples of 4 (element-wise stores of the cluster reduction)."""
     w = synth.weights_f32(n, k, seed=11 + n)
     x = synth.activations_bf16(t, k, seed=12 + t)
     ref = oracle.pack(q.BF16, w.numpy())
@@ -272,8 +274,9 @@ def test_gemv_bf16_weights_prefill_ragged_n(n, k, t, y_dtype):
 @pytest.mark.parametrize("t", [8192, 40000])
 def test_gemv_bf16_gdn_ab_full_size_sampled(t):
     """The GDN a/b projection 96 x 5120 at an 8192-token prefill chunk (K split
-    three ways) and at 40000 tokens (one part per tile): sampled tokens,
-    always the first and the last (ragged) tile."""
+    over a cluster of CTAs, reduced through distributed shared memory) and at
+    40000 tokens (one part per tile): sampled tokens, always the first and the
+    last (ragged) tile."""
     n, k = 96, 5120
     w = synth.weights_f32(n, k, seed=synth.seed_for(5, 0), device=DEV)
     x = synth.activations_bf16(t, k, seed=synth.seed_for(5, 1), device=DEV)
