@@ -113,16 +113,21 @@ __global__ void __launch_bounds__(512) quantize_act_kernel(const uint16_t* __res
   const int64_t total = groups * 8;  // 8 lanes per group
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   // whole warps iterate together (the shuffles need every lane); two 16-byte
-  // loads per thread in flight
-  for (int64_t wbase = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); wbase < total;
-       wbase += 2 * stride) {
+  // loads per thread per step, and the next step's two loads are issued before
+  // this step's codes are computed (four in flight)
+  int64_t wbase = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  auto load = [&](int64_t i) {
+    return i < total ? __ldcs((const uint4*)(x + i * 8)) : make_uint4(0, 0, 0, 0);
+  };
+  uint4 r0 = load(wbase + lane), r1 = load(wbase + stride + lane);
+  for (; wbase < total; wbase += 2 * stride) {
     const int64_t i0 = wbase + lane, i1 = wbase + stride + lane;
     const bool v0 = i0 < total, v1 = i1 < total;  // total % 8 == 0: a group is valid or not as a whole
-    uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
-    if (v0) r0 = __ldcs((const uint4*)(x + i0 * 8));
-    if (v1) r1 = __ldcs((const uint4*)(x + i1 * 8));
+    const uint4 n0 = load(i0 + 2 * stride), n1 = load(i1 + 2 * stride);
     quantize_group8(r0, lane, v0, i0, xq, xs);
     if (__any_sync(0xffffffffu, v1)) quantize_group8(r1, lane, v1, i1, xq, xs);
+    r0 = n0;
+    r1 = n1;
   }
 }
 

@@ -63,6 +63,8 @@ struct B16Args {
   int out_dtype;      // QLIN_OUT_BF16 / QLIN_OUT_F32
 };
 
+constexpr int kMaxParts = 16;  // non-portable cluster size; 8 where the device refuses 16
+
 // The FP32 partial of a CTA in its shared memory: [MT * 128 tokens][NP + 4]
 // (the 4-float pad keeps the 16-byte row writes of a warp on distinct banks).
 template <int NP>
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(B16_THREADS, 1)
   };
 
   if (warp == B16_WTMA) {
+    const uint64_t pol_x = l2_evict_first(), pol_w = l2_evict_last();  // x streams once; W serves every tile
     int slot = 0, phase = 0, issued = 0;
     for (int kb = kb0; kb < kb1; ++kb) {
       if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait(&empty[slot], (uint32_t)(phase ^ 1)))) {
@@ -147,8 +150,8 @@ __global__ void __launch_bounds__(B16_THREADS, 1)
         mbar_arrive_expect_tx(&full[slot], C::STAGE);
 #pragma unroll
         for (int m = 0; m < MT; ++m)
-          tma_load_2d(st + m * C::A_SUB, &tm_x, &full[slot], kb * B16_BK, (tile * MT + m) * B16_BM);
-        tma_load_2d(st + C::A_BYTES, &tm_w, &full[slot], kb * B16_BK, 0);
+          tma_load_2d_hint(st + m * C::A_SUB, &tm_x, &full[slot], kb * B16_BK, (tile * MT + m) * B16_BM, pol_x);
+        tma_load_2d_hint(st + C::A_BYTES, &tm_w, &full[slot], kb * B16_BK, 0, pol_w);
       }
       __syncwarp();
       ++issued;
@@ -271,13 +274,21 @@ __global__ void __launch_bounds__(B16_THREADS, 1)
       const int64_t tok = (int64_t)tile * MT * B16_BM + ltok;
       if (tok >= args.t || col >= args.n) continue;
       const uint32_t off = (uint32_t)(ltok * red_stride<NP>() + col) * 4u;
-      float4 acc = ld_dsmem_v4(map_to_rank(red_s + off, 0));
-      for (int p = 1; p < P; ++p) {
-        const float4 v = ld_dsmem_v4(map_to_rank(red_s + off, (uint32_t)p));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+      // all P loads in flight at once (one distributed-shared-memory latency),
+      // then the sum in part order
+      float4 v[kMaxParts];
+#pragma unroll
+      for (int p = 0; p < kMaxParts; ++p)
+        if (p < P) v[p] = ld_dsmem_v4(map_to_rank(red_s + off, (uint32_t)p));
+      float4 acc = v[0];
+#pragma unroll
+      for (int p = 1; p < kMaxParts; ++p) {
+        if (p < P) {
+          acc.x += v[p].x;
+          acc.y += v[p].y;
+          acc.z += v[p].z;
+          acc.w += v[p].w;
+        }
       }
       const int64_t o = tok * args.n + col;
       if (vec) {
@@ -324,7 +335,6 @@ int np_of(int64_t n) { return n <= 64 ? 64 : n <= 96 ? 96 : n <= 128 ? 128 : 256
 // N = 256 (the partial of two sub-tiles would not fit the stage buffers).
 int mt_of(int64_t t, int np) { return t >= 1024 && np <= 128 ? 2 : 1; }
 
-constexpr int kMaxParts = 16;  // non-portable cluster size; 8 where the device refuses 16
 
 // Clusters of `p` CTAs that can be resident at once on this device (cached per
 // device and configuration); 0 when the device refuses the cluster size.

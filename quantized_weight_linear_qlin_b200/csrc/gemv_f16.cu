@@ -319,11 +319,12 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     // ---- producer.  The codes of the first stages go out before the wait for
     // the activation conversion (programmatic dependent launch); their
     // activation boxes follow once it has completed.
+    const uint64_t pol_w = l2_evict_first(), pol_x = l2_evict_last();  // codes stream once; x serves every CTA
     const int npre = nunits < NS ? nunits : NS;
     auto issue_x = [&](int s, int ch) {
 #pragma unroll
       for (int b = 0; b < L::XBOXES; ++b)
-        tma_load_2d(stage(s) + L::OFF_X + b * TP * 128, &tm_x, &full[s], ch * KC + b * 64, 0);
+        tma_load_2d_hint(stage(s) + L::OFF_X + b * TP * 128, &tm_x, &full[s], ch * KC + b * 64, 0, pol_x);
     };
     Ring ring{0, 0};
     int tile = tile0, ch = ch0;
@@ -340,8 +341,8 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         mbar_arrive_expect_tx(&full[s], L::TMA_BYTES);
 #pragma unroll
         for (int b = 0; b < UB; ++b)
-          tma_load_2d(st + b * BOX_BYTES, &tm_codes, &full[s], (ch * UB + b) * 128, tile * 128);
-        if (Tr::PER_GROUP) tma_load_2d(st + L::OFF_SC, &tm_sc, &full[s], (ch * L::GPC) & ~7, tile * 128);
+          tma_load_2d_hint(st + b * BOX_BYTES, &tm_codes, &full[s], (ch * UB + b) * 128, tile * 128, pol_w);
+        if (Tr::PER_GROUP) tma_load_2d_hint(st + L::OFF_SC, &tm_sc, &full[s], (ch * L::GPC) & ~7, tile * 128, pol_w);
         if (cu >= npre) issue_x(s, ch);
       }
       __syncwarp();

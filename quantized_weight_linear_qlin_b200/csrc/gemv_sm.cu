@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
   };
 
   if (warp == 0) {
+    const uint64_t pol_w = l2_evict_first(), pol_x = l2_evict_last();  // codes stream once; x serves every CTA
     int issued = 0;
     Ring ring{0, 0};
     int tile = tile0, ch = ch0;
@@ -144,11 +145,11 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
         mbar_arrive_expect_tx(&full[s], C::TMA_BYTES);
 #pragma unroll
         for (int b = 0; b < UBS; ++b)
-          tma_load_2d(st + b * BOX_BYTES, &tm_codes, &full[s], (ch * UBS + b) * 128, tile * 128);
-        if (Tr::HIB) tma_load_2d(st + C::OFF_HIB, &tm_hib, &full[s], ch * UBS * Tr::HROW, tile * 128);
+          tma_load_2d_hint(st + b * BOX_BYTES, &tm_codes, &full[s], (ch * UBS + b) * 128, tile * 128, pol_w);
+        if (Tr::HIB) tma_load_2d_hint(st + C::OFF_HIB, &tm_hib, &full[s], ch * UBS * Tr::HROW, tile * 128, pol_w);
 #pragma unroll
         for (int b = 0; b < C::XBOXES; ++b)
-          tma_load_2d(st + C::OFF_X + b * T * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0);
+          tma_load_2d_hint(st + C::OFF_X + b * T * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0, pol_x);
       }
       if constexpr (Tr::PER_GROUP) {
         const __half* src = (const __half*)args.scales + ch * GPC;

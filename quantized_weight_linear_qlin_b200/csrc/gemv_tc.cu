@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // lane 0 issues the TMA copies; all 32 lanes copy the unit's group scales
     // (SC_ROW bytes per row) with cp.async, tracked by the same barrier.
+    const uint64_t pol_w = l2_evict_first(), pol_x = l2_evict_last();  // codes stream once; x serves every CTA
     int issued = 0;
     Ring ring{0, 0};
     int tile = tile0, ch = ch0;
@@ -203,11 +204,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive_expect_tx(&full[s], L::TMA_BYTES);
 #pragma unroll
         for (int b = 0; b < UB; ++b)
-          tma_load_2d(codes_s + (s * UB + b) * BOX_BYTES, &tm_codes, &full[s], (ch * UB + b) * 128, tile * 128);
-        if (Tr::HIB) tma_load_2d(hib_s + s * L::HIB_BYTES, &tm_hib, &full[s], ch * UB * Tr::HROW, tile * 128);
+          tma_load_2d_hint(codes_s + (s * UB + b) * BOX_BYTES, &tm_codes, &full[s], (ch * UB + b) * 128, tile * 128,
+                           pol_w);
+        if (Tr::HIB)
+          tma_load_2d_hint(hib_s + s * L::HIB_BYTES, &tm_hib, &full[s], ch * UB * Tr::HROW, tile * 128, pol_w);
 #pragma unroll
         for (int b = 0; b < L::XBOXES; ++b)
-          tma_load_2d(x_s + s * L::X_BYTES + b * TP * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0);
+          tma_load_2d_hint(x_s + s * L::X_BYTES + b * TP * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0, pol_x);
       }
       if constexpr (Tr::PER_GROUP) {
         const __half* src = (const __half*)args.scales + ch * GPC;

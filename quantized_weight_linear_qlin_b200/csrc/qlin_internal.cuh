@@ -158,6 +158,31 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+// L2 eviction priorities for TMA loads: data that this launch reads once
+// (weight codes streamed by the projections, the activations of a prefill
+// chunk) goes first, so that it does not push out lines that are still wanted
+// (dirty lines of earlier kernels, operands that other CTAs read again);
+// operands that every CTA reads (x of a decode step, the small BF16 weight of
+// a prefill projection) go last.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+// tma_load_2d with an L2 cache policy from l2_evict_first / l2_evict_last.
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                                 int y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
 
 // Asynchronous 8-byte global -> shared copy (non-bulk), and an mbarrier arrival
 // that fires once all of this thread's earlier cp.async copies have landed (the
