@@ -116,8 +116,16 @@ __global__ void __launch_bounds__(512) quantize_act_kernel(const uint16_t* __res
   // loads per thread per step, and the next step's two loads are issued before
   // this step's codes are computed (four in flight)
   int64_t wbase = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  // x is read once: its lines go first when L2 needs room (they do not push
+  // out the dirty lines of earlier kernels, which would cost a write-back)
+  const uint64_t pol = l2_evict_first();
   auto load = [&](int64_t i) {
-    return i < total ? __ldcs((const uint4*)(x + i * 8)) : make_uint4(0, 0, 0, 0);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (i < total)
+      asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "l"(x + i * 8), "l"(pol));
+    return v;
   };
   uint4 r0 = load(wbase + lane), r1 = load(wbase + stride + lane);
   for (; wbase < total; wbase += 2 * stride) {
@@ -934,7 +942,9 @@ int launch_quantize_act(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, flo
   const int64_t groups = t * (k / 64);
   const int64_t threads = groups * 8;
   int64_t blocks = (threads + 511) / 512;
-  const int64_t cap = (int64_t)ex.num_sms * 8;
+  // four 512-thread blocks per SM (two are resident at a time): measured
+  // faster than one resident wave or than eight blocks per SM
+  const int64_t cap = (int64_t)ex.num_sms * 4;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   quantize_act_kernel<<<(unsigned)blocks, 512, 0, ex.stream>>>(x, groups, xq, xs);
