@@ -340,9 +340,10 @@ def run_ours(args, dist):
 
     # ---- e2e: through the public API with pinned host buffers.  Each step's
     # eight activation tensors go up in one host-to-device copy and its eight
-    # results come back in one device-to-host copy, on a copy stream: the
-    # inputs of step i+1 (double-buffered) and the results of step i move while
-    # step i+1 computes, as a serving loop would overlap them.
+    # results come back in one device-to-host copy, each direction on a copy
+    # stream of its own (the two directions run at once): the inputs of step
+    # i+1 (double-buffered) move while step i computes, and the results of
+    # step i while step i+1 computes, as a serving loop would overlap them.
     xs_list = [x for t in T_LIST for x in (xs_gu[t], xs_dn[t])]
     ys_list = [y for t in T_LIST for y in (ys_gu[t], ys_dn[t])]
     hx_all = torch.cat([x.reshape(-1) for x in xs_list]).cpu().pin_memory()
@@ -363,31 +364,35 @@ def run_ours(args, dist):
     h2d = hx_all.numel() * 2
     d2h = hy_all.numel() * 2
     main = torch.cuda.current_stream()
-    side = torch.cuda.Stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     h2d_done = [torch.cuda.Event() for _ in range(2)]
     comp_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
 
     def e2e_run(n):
-        side.wait_stream(main)
-        with torch.cuda.stream(side):
-            dx_all[0].copy_(hx_all, non_blocking=True)
-        h2d_done[0].record(side)
+        up.wait_stream(main)
+        down.wait_stream(main)
         for i in range(n):
             b = i & 1
+            if i >= 2:
+                up.wait_event(comp_done[b])  # step i-2 has read input buffer b
+            with torch.cuda.stream(up):
+                dx_all[b].copy_(hx_all, non_blocking=True)
+            h2d_done[b].record(up)
             main.wait_event(h2d_done[b])
+            if i >= 2:
+                main.wait_event(d2h_done[b])  # step i-2's results have left output buffer b
             for ti, t in enumerate(T_LIST):
                 gu, dn = copies[ti]
                 q.qlin_gemv(gu, dxv[b][2 * ti], dyv[b][2 * ti], q.OUT_BF16, workspace=ws)
                 q.qlin_gemv(dn, dxv[b][2 * ti + 1], dyv[b][2 * ti + 1], q.OUT_BF16, workspace=ws)
             comp_done[b].record(main)
-            side.wait_event(comp_done[b])  # step i's results, and its input buffer is free
-            with torch.cuda.stream(side):
+            down.wait_event(comp_done[b])
+            with torch.cuda.stream(down):
                 hy_all.copy_(dy_all[b], non_blocking=True)
-                if i + 1 < n:
-                    dx_all[1 - b].copy_(hx_all, non_blocking=True)
-            if i + 1 < n:
-                h2d_done[1 - b].record(side)
-        main.wait_stream(side)
+            d2h_done[b].record(down)
+        main.wait_stream(up)
+        main.wait_stream(down)
 
     e2e_run(args.warmup)
     torch.cuda.synchronize()
