@@ -201,6 +201,11 @@ QLIN_API int qlin_gemv_workspace_bytes(const qlin_weights* w, int64_t t, size_t*
  * After a call that reported QLIN_ERR_TIMEOUT its split-tile counters may be
  * left non-zero: zero-fill the workspace again before its next use
  * (qlin_gemv_noalloc clears its own counters on every call).
+ * Ordering: the kernels are launched with programmatic dependent launch, so
+ * they may start, and read the packed weights, while the kernel ahead of them
+ * on `stream` is still finishing (when that kernel allows it); x, y and the
+ * workspace are touched only once it has completed.  The weights must not be
+ * written by a kernel that is still running.
  * Accuracy: |y - y_ref| <= 1e-3 * sum_k |w||x| per element (plus the BF16
  * output rounding).  ["NInfer int8-prefill artifact for the RTX 4090",
  * "What changes": decode keeps the BF16 route; "...NVFP4-NInferV3", "How it

@@ -123,6 +123,9 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
     if (Tr::HIB) tma_prefetch_desc(&tm_hib);
   }
   __syncthreads();
+  // the next kernel on the stream may be scheduled as this one's CTAs leave;
+  // it waits (griddepcontrol.wait) before it touches anything this one writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   auto abort_now = [&]() {
     *abort_flag = 1;
@@ -130,7 +133,11 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
   };
 
   if (warp == 0) {
+    // the weights of the first NS units (codes, planes, scales: never written
+    // by the kernels of a decode step) go out before the wait for the kernel
+    // launched ahead of this one; x, which that kernel may produce, after it
     const uint64_t pol_w = l2_evict_first(), pol_x = l2_evict_last();  // codes stream once; x serves every CTA
+    const int npre = nunits < NS ? nunits : NS;
     int issued = 0;
     Ring ring{0, 0};
     int tile = tile0, ch = ch0;
@@ -147,9 +154,11 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
         for (int b = 0; b < UBS; ++b)
           tma_load_2d_hint(st + b * BOX_BYTES, &tm_codes, &full[s], (ch * UBS + b) * 128, tile * 128, pol_w);
         if (Tr::HIB) tma_load_2d_hint(st + C::OFF_HIB, &tm_hib, &full[s], ch * UBS * Tr::HROW, tile * 128, pol_w);
+        if (cu >= npre) {
 #pragma unroll
-        for (int b = 0; b < C::XBOXES; ++b)
-          tma_load_2d_hint(st + C::OFF_X + b * T * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0, pol_x);
+          for (int b = 0; b < C::XBOXES; ++b)
+            tma_load_2d_hint(st + C::OFF_X + b * T * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0, pol_x);
+        }
       }
       if constexpr (Tr::PER_GROUP) {
         const __half* src = (const __half*)args.scales + ch * GPC;
@@ -171,6 +180,19 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
         ch = 0;
         ++tile;
       }
+      if (cu == npre - 1) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (lane == 0) {
+          // the activation boxes of the first npre units (stages 0..npre-1)
+          for (int c = 0; c < npre; ++c) {
+            const int chc = (int)((ch0 + c) % cpt);
+            uint8_t* stc = base + c * C::STAGE;
+#pragma unroll
+            for (int b = 0; b < C::XBOXES; ++b)
+              tma_load_2d_hint(stc + C::OFF_X + b * T * 128, &tm_x, &full[c], chc * C::KC + b * 64, 0, pol_x);
+          }
+        }
+      }
     }
     if (lane == 0) {
       Ring r2{0, 0};
@@ -181,6 +203,8 @@ __global__ void __launch_bounds__(SmCfg<FMT, T>::THREADS, 1)
     }
   } else {
     // ---- compute warps: row r of the tile, part h of the unit's groups
+    // (y and the split-tile workspace may still be in use by the kernel ahead)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int cw = warp - 1;
     const int r = cw * RPW + (lane % RPW);
     const int h = lane / RPW;
@@ -342,8 +366,17 @@ int launch_t(const CUtensorMap& mc, const CUtensorMap& mh, const CUtensorMap& mx
   auto kern = gemv_sm_kernel<FMT, T>;
   const cudaError_t e = set_smem_once<gemv_sm_kernel<FMT, T>>((int)C::SMEM);
   if (e != cudaSuccess) return cuda_status(e);
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(mc, mh, mx, a);
-  return cuda_status(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, mc, mh, mx, a));
 }
 
 template <int FMT>

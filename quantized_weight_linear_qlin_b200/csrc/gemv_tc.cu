@@ -181,6 +181,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the next kernel on the stream may be scheduled as this one's CTAs leave;
+  // it waits (griddepcontrol.wait) before it touches anything this one writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   auto abort_now = [&]() {
     *abort_flag = 1;
@@ -189,8 +192,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     // lane 0 issues the TMA copies; all 32 lanes copy the unit's group scales
-    // (SC_ROW bytes per row) with cp.async, tracked by the same barrier.
+    // (SC_ROW bytes per row) with cp.async, tracked by the same barrier.  The
+    // weights of the first NS units (codes, planes, scales: never written by
+    // the kernels of a decode step) go out before the wait for the kernel
+    // launched ahead of this one; x, which that kernel may produce, after it.
     const uint64_t pol_w = l2_evict_first(), pol_x = l2_evict_last();  // codes stream once; x serves every CTA
+    const int npre = nunits < NS ? nunits : NS;
     int issued = 0;
     Ring ring{0, 0};
     int tile = tile0, ch = ch0;
@@ -208,9 +215,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                            pol_w);
         if (Tr::HIB)
           tma_load_2d_hint(hib_s + s * L::HIB_BYTES, &tm_hib, &full[s], ch * UB * Tr::HROW, tile * 128, pol_w);
+        if (cu >= npre) {
 #pragma unroll
-        for (int b = 0; b < L::XBOXES; ++b)
-          tma_load_2d_hint(x_s + s * L::X_BYTES + b * TP * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0, pol_x);
+          for (int b = 0; b < L::XBOXES; ++b)
+            tma_load_2d_hint(x_s + s * L::X_BYTES + b * TP * 128, &tm_x, &full[s], ch * C::KC + b * 64, 0, pol_x);
+        }
       }
       if constexpr (Tr::PER_GROUP) {
         const __half* src = (const __half*)args.scales + ch * GPC;
@@ -231,6 +240,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (++ch == cpt) {
         ch = 0;
         ++tile;
+      }
+      if (cu == npre - 1) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (lane == 0) {
+          // the activation boxes of the first npre units (stages 0..npre-1)
+          for (int c = 0; c < npre; ++c) {
+            const int chc = (int)((ch0 + c) % cpt);
+#pragma unroll
+            for (int b = 0; b < L::XBOXES; ++b)
+              tma_load_2d_hint(x_s + c * L::X_BYTES + b * TP * 128, &tm_x, &full[c], chc * C::KC + b * 64, 0,
+                               pol_x);
+          }
+        }
       }
     }
     if (lane == 0)
@@ -360,6 +382,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       ring.next(NS);
     }
   } else if (warp >= W_EPI0) {
+    // y and the split-tile workspace may still be in use by the kernel ahead
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int et = threadIdx.x - W_EPI0 * 32;  // 0..127
@@ -551,8 +575,17 @@ int launch_tp(const CUtensorMap& mc, const CUtensorMap& mh, const CUtensorMap& m
   auto kern = gemv_tc_kernel<FMT, TP>;
   const cudaError_t e = set_smem_once<gemv_tc_kernel<FMT, TP>>((int)C::SMEM);
   if (e != cudaSuccess) return cuda_status(e);
-  kern<<<grid, THREADS, C::SMEM, st>>>(mc, mh, mx, a);
-  return cuda_status(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, mc, mh, mx, a));
 }
 
 template <int FMT>
