@@ -321,7 +321,12 @@ int qlin_gemv(const qlin_weights* w, const uint16_t* x_bf16, int64_t t, void* y,
 
 int qlin_gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, size_t* bytes) {
   if (!bytes || t <= 0 || n <= 0 || k <= 0 || k % 64) return QLIN_ERR_INVALID_ARG;
-  *bytes = gemm_a8_workspace_bytes(t, n, k, 0);
+  // the stream-K partials are sized for the current device's SMs (256 when no
+  // device is visible, which covers any current part)
+  Exec e;
+  const int sms = make_exec(nullptr, &e) == QLIN_OK ? e.num_sms : 256;
+  (void)cudaGetLastError();
+  *bytes = gemm_a8_workspace_bytes(t, n, k, sms);
   return QLIN_OK;
 }
 

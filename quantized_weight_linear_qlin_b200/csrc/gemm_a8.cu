@@ -202,6 +202,8 @@ struct GemmArgs {
   int64_t tiles_t;       // token tiles
   int64_t tiles;         // row tiles x token tiles
   int y_dtype;
+  float* partials;       // stream-K split tiles: [CTAs][2][BN tokens][BM rows] FP32
+  int* counters;         // stream-K split tiles: [tiles][epilogue warps], zero at launch
 };
 
 template <class SM>
@@ -675,7 +677,12 @@ struct XSmem {
 
 template <int BITS>
 __global__ void expand_i8_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ hib,
-                                 int64_t n, int64_t k, int8_t* __restrict__ out) {
+                                 int64_t n, int64_t k, int8_t* __restrict__ out, int* __restrict__ counters,
+                                 int64_t ncounters) {
+  // the GEMM's split-tile counters start the call at zero
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < ncounters;
+       i += (int64_t)gridDim.x * blockDim.x)
+    counters[i] = 0;
   const int64_t ng = k / 64;
   for (int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; item < n * ng;
        item += (int64_t)gridDim.x * blockDim.x) {
@@ -714,7 +721,18 @@ __global__ void __launch_bounds__(X_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ng = args.k / 64;
   const int nchunks = (int)(args.k / X_BK);
-  const int64_t my_tiles = (args.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+  // Whole tiles in full waves (tile = CTA + round * CTAs: the CTAs that run at
+  // the same time share weight row tiles, which L2 then serves), then the
+  // tiles left over after the last full wave split evenly over all CTAs by
+  // their (tile, K chunk) iterations (stream-K), so that no SM idles through a
+  // partial last wave.
+  // (32-bit counts: tiles x chunks < 2^31 is checked on the host)
+  const int P = (int)gridDim.x, ntiles = (int)args.tiles;
+  const int rounds = ntiles / P, dp_tiles = rounds * P;
+  const int iters = (ntiles - dp_tiles) * nchunks;  // stream-K iterations
+  const int it0 = (int)((int64_t)blockIdx.x * iters / P), it1 = (int)(((int64_t)blockIdx.x + 1) * iters / P);
+  const int dp_jobs = rounds * nchunks;
+  const int njobs = dp_jobs + (it1 - it0);  // this CTA's (tile, chunk) steps
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < X_NS; ++s) {
@@ -748,10 +766,23 @@ __global__ void __launch_bounds__(X_THREADS, 1)
     int issued = 0;
     Ring ring{0, 0};
     bool ok = true;
-    for (int64_t it = 0; it < my_tiles && ok; ++it) {
-      const int64_t tile = blockIdx.x + it * gridDim.x;
-      const int64_t n0 = (tile / args.tiles_t) * BM, t0 = (tile % args.tiles_t) * BN;
-      for (int kc = 0; kc < nchunks; ++kc) {
+    // the steps' tile and K chunk, advanced incrementally (no division per step)
+    int tile = (int)blockIdx.x, kc = 0;
+    if (dp_jobs == 0) {
+      tile = dp_tiles + it0 / nchunks;
+      kc = it0 - (it0 / nchunks) * nchunks;
+    }
+    const int tiles_t = (int)args.tiles_t;
+    int rt = tile / tiles_t, tt = tile - rt * tiles_t;  // row tile, token tile
+    for (int j = 0; j < njobs && ok; ++j) {
+      if (j == dp_jobs && j > 0) {  // from the full waves into the stream-K range
+        tile = dp_tiles + it0 / nchunks;
+        kc = it0 - (it0 / nchunks) * nchunks;
+        rt = tile / tiles_t;
+        tt = tile - rt * tiles_t;
+      }
+      const int64_t n0 = (int64_t)rt * BM, t0 = (int64_t)tt * BN;
+      {
         const int s = ring.slot;
         if (!__all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.empty[s], (uint32_t)(ring.phase ^ 1)))) {
           if (lane == 0) set_abort(sm, args.dev_status);
@@ -778,6 +809,12 @@ __global__ void __launch_bounds__(X_THREADS, 1)
         ++issued;
         ring.next(X_NS);
       }
+      if (++kc == nchunks) {  // next tile: the next wave's, or the next one in the range
+        kc = 0;
+        tile += j < dp_jobs ? P : 1;
+        rt = tile / tiles_t;
+        tt = tile - rt * tiles_t;
+      }
     }
     if (lane == 0) {
       Ring r2{0, 0};
@@ -790,8 +827,8 @@ __global__ void __launch_bounds__(X_THREADS, 1)
     const uint32_t idesc = idesc_i8(BM, BN);
     Ring ring{0, 0}, dr{0, 0};
     bool ok = true;
-    for (int64_t it = 0; it < my_tiles && ok; ++it) {
-      for (int kc = 0; kc < nchunks && ok; ++kc) {
+    for (int j = 0; j < njobs && ok; ++j) {
+      {
         const int s = ring.slot;
         ok = __all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.full[s], (uint32_t)ring.phase));
         if (!ok) break;
@@ -824,16 +861,17 @@ __global__ void __launch_bounds__(X_THREADS, 1)
     const int row = quarter * 32 + lane;
     const int col0 = cblk * 32;
     const uint32_t lane_ofs = (uint32_t)(quarter * 32) << 16;
+    // the split-tile counters come from the kernels launched just before
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     Ring ring{0, 0}, dr{0, 0};
     bool ok = true;
-    for (int64_t it = 0; it < my_tiles && ok; ++it) {
-      const int64_t tile = blockIdx.x + it * gridDim.x;
-      const int64_t n0 = (tile / args.tiles_t) * BM, t0 = (tile % args.tiles_t) * BN;
+    // y (this thread's row, 32 tokens) of one tile over chunks [kc0, kc1)
+    auto run = [&](int tile, int kc0, int kc1, float2 (&y2)[16]) {
+      const int64_t n0 = (int64_t)(tile / (int)args.tiles_t) * BM, t0 = (int64_t)(tile % (int)args.tiles_t) * BN;
       const int64_t grow = n0 + row;
-      float2 y2[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) y2[j] = make_float2(0.0f, 0.0f);
-      for (int kc = 0; kc < nchunks && ok; ++kc) {
+      for (int kc = kc0; kc < kc1 && ok; ++kc) {
         const int s = ring.slot;
         // the stage's scales have landed once its barrier completed (acquire)
         ok = __all_sync(0xffffffffu, !aborted(sm) && mbar_wait(&sm.full[s], (uint32_t)ring.phase));
@@ -876,25 +914,76 @@ __global__ void __launch_bounds__(X_THREADS, 1)
         if (lane == 0) mbar_arrive(&sm.empty[s]);  // the stage's scales are consumed
         ring.next(X_NS);
       }
-      if (!ok) {
-        set_abort(sm, args.dev_status);
-        break;
-      }
-      if (grow < args.n) {
-        const int jmax = (int)min((int64_t)32, args.t - (t0 + col0));
-        const int64_t base = (t0 + col0) * args.n + grow;
+    };
+    auto store = [&](int tile, const float2 (&y2)[16]) {
+      const int64_t n0 = (int64_t)(tile / (int)args.tiles_t) * BM, t0 = (int64_t)(tile % (int)args.tiles_t) * BN;
+      const int64_t grow = n0 + row;
+      if (grow >= args.n) return;
+      const int jmax = (int)min((int64_t)32, args.t - (t0 + col0));
+      const int64_t base = (t0 + col0) * args.n + grow;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j < jmax) {
-            const float v = (j & 1) ? y2[j >> 1].y : y2[j >> 1].x;
-            if (args.y_dtype == QLIN_OUT_F32)
-              ((float*)args.y)[base + (int64_t)j * args.n] = v;
-            else
-              ((__nv_bfloat16*)args.y)[base + (int64_t)j * args.n] = __float2bfloat16_rn(v);
+      for (int j = 0; j < 32; ++j) {
+        if (j < jmax) {
+          const float v = (j & 1) ? y2[j >> 1].y : y2[j >> 1].x;
+          if (args.y_dtype == QLIN_OUT_F32)
+            ((float*)args.y)[base + (int64_t)j * args.n] = v;
+          else
+            ((__nv_bfloat16*)args.y)[base + (int64_t)j * args.n] = __float2bfloat16_rn(v);
+        }
+      }
+    };
+    float2 y2[16];
+    // full waves: whole tiles
+    for (int r = 0; r < rounds && ok; ++r) {
+      const int tile = (int)blockIdx.x + r * P;
+      run(tile, 0, nchunks, y2);
+      if (!ok) break;
+      store(tile, y2);
+    }
+    // the stream-K range: segments of whole tiles, or the first and last tile
+    // of the range shared with neighbouring CTAs
+    for (int g = it0; g < it1 && ok;) {
+      const int tile = dp_tiles + g / nchunks;
+      const int kc0 = g - (g / nchunks) * nchunks;
+      const int kc1 = min(nchunks, kc0 + (it1 - g));
+      g += kc1 - kc0;
+      run(tile, kc0, kc1, y2);
+      if (!ok) break;
+      if (kc0 != 0 || kc1 != nchunks) {
+        // a split tile: publish this part ([token][row] FP32, slot 0 for the
+        // CTA's first tile, 1 for its last); the warp that arrives last for
+        // this block of the tile sums every part in CTA order and writes y
+        const int ew = warp - X_WEPI0;
+        const int slot = tile == dp_tiles + it0 / nchunks ? 0 : 1;
+        float* mine = args.partials + ((int64_t)blockIdx.x * 2 + slot) * (BM * BN) + (int64_t)col0 * BM + row;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mine[j * BM] = (j & 1) ? y2[j >> 1].y : y2[j >> 1].x;
+        __threadfence();
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atomicAdd(&args.counters[(int64_t)tile * X_NEPI + ew], 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        // the CTAs that own the tile's first and last stream-K iterations
+        const int64_t g0 = (int64_t)(tile - dp_tiles) * nchunks;
+        const int i_first = (int)(((g0 + 1) * P - 1) / iters);
+        const int i_last = (int)(((g0 + nchunks) * P - 1) / iters);
+        if (old != i_last - i_first) continue;
+        __threadfence();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) y2[j] = make_float2(0.0f, 0.0f);
+        for (int i = i_first; i <= i_last; ++i) {
+          const int si = tile == dp_tiles + (int)((int64_t)i * iters / P) / nchunks ? 0 : 1;
+          const float* part = args.partials + ((int64_t)i * 2 + si) * (BM * BN) + (int64_t)col0 * BM + row;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            y2[j].x += __ldcg(part + (2 * j) * BM);
+            y2[j].y += __ldcg(part + (2 * j + 1) * BM);
           }
         }
       }
+      store(tile, y2);
     }
+    if (!ok) set_abort(sm, args.dev_status);
   }
 
   // Every group sum's completion was observed by the epilogue before this
@@ -919,23 +1008,28 @@ __global__ void __launch_bounds__(X_THREADS, 1)
 // [N][K] (each part 256-byte aligned).  A workspace too small for the last
 // part runs the kernel that expands the codes in tensor memory instead.
 struct A8Ws {
-  size_t xq, xs, w8, total, act_total;
+  size_t xq, xs, w8, counters, partials, total, act_total;
+  int64_t ncounters;
 };
-static A8Ws a8_ws(int64_t t, int64_t n, int64_t k) {
+static size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+static A8Ws a8_ws(int64_t t, int64_t n, int64_t k, int num_sms) {
   A8Ws L;
   L.xq = 0;
-  L.xs = ((size_t)t * k + 255) / 256 * 256;
+  L.xs = up256((size_t)t * k);
   L.act_total = L.xs + (size_t)t * (k / 64) * sizeof(float);
-  L.w8 = (L.act_total + 255) / 256 * 256;
-  L.total = L.w8 + (size_t)n * k;
+  L.w8 = up256(L.act_total);
+  const int64_t tiles = ((n + BM - 1) / BM) * ((t + BN - 1) / BN);
+  L.ncounters = tiles * X_NEPI;
+  L.counters = up256(L.w8 + (size_t)n * k);
+  L.partials = up256(L.counters + (size_t)L.ncounters * sizeof(int));
+  L.total = L.partials + (size_t)(num_sms > 0 ? num_sms : 1) * 2 * BM * BN * sizeof(float);
   return L;
 }
 
 size_t gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, int num_sms) {
-  (void)num_sms;
-  return a8_ws(t, n, k).total;
+  return a8_ws(t, n, k, num_sms).total;
 }
-size_t gemm_a8_act_workspace_bytes(int64_t t, int64_t k) { return a8_ws(t, 0, k).act_total; }
+size_t gemm_a8_act_workspace_bytes(int64_t t, int64_t k) { return a8_ws(t, 0, k, 1).act_total; }
 
 int launch_quantize_act(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* xs,
                         const Exec& ex) {
@@ -993,8 +1087,11 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
                    int64_t t, void* y, int y_dtype, uint32_t flags, int32_t* sums_dbg,
                    const Exec& ex) {
   const int64_t n = w.n, k = w.k;
-  const A8Ws wl = a8_ws(t, n, k);
-  const bool expanded = ex.workspace != nullptr && ex.workspace_bytes >= wl.total;
+  const A8Ws wl = a8_ws(t, n, k, ex.num_sms);
+  // (the expanded-weight kernel counts its (tile, K chunk) steps in 32 bits)
+  const int64_t xtiles = ((n + BM - 1) / BM) * ((t + BN - 1) / BN);
+  const bool expanded = ex.workspace != nullptr && ex.workspace_bytes >= wl.total &&
+                        xtiles * (k / X_BK) < (int64_t)INT32_MAX;
   const int bits = w.fmt == QLIN_Q3_G64 ? 3 : w.fmt == QLIN_Q4_G64 ? 4 : w.fmt == QLIN_Q5_G64 ? 5 : 6;
   int8_t* w8 = expanded ? (int8_t*)((uint8_t*)ex.workspace + wl.w8) : nullptr;
   if (expanded) {
@@ -1003,11 +1100,12 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
     const int64_t blocks = std::min<int64_t>((items + 255) / 256, (int64_t)ex.num_sms * 16);
     const uint8_t* c = (const uint8_t*)w.codes;
     const uint8_t* h = (const uint8_t*)w.hibits;
+    int* cnt = (int*)((uint8_t*)ex.workspace + wl.counters);
     switch (bits) {
-      case 3: expand_i8_kernel<3><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8); break;
-      case 4: expand_i8_kernel<4><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8); break;
-      case 5: expand_i8_kernel<5><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8); break;
-      default: expand_i8_kernel<6><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8); break;
+      case 3: expand_i8_kernel<3><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8, cnt, wl.ncounters); break;
+      case 4: expand_i8_kernel<4><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8, cnt, wl.ncounters); break;
+      case 5: expand_i8_kernel<5><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8, cnt, wl.ncounters); break;
+      default: expand_i8_kernel<6><<<(unsigned)blocks, 256, 0, ex.stream>>>(c, h, n, k, w8, cnt, wl.ncounters); break;
     }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e);
@@ -1041,7 +1139,10 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
     args.tiles_t = (t + BN - 1) / BN;
     args.tiles = args.tiles_t * ((n + BM - 1) / BM);
     args.y_dtype = y_dtype;
-    const int grid = (int)std::min<int64_t>(args.tiles, ex.num_sms);
+    args.partials = (float*)((uint8_t*)ex.workspace + wl.partials);
+    args.counters = (int*)((uint8_t*)ex.workspace + wl.counters);
+    // stream-K: every SM takes an equal share of the (tile, K chunk) iterations
+    const int grid = (int)std::min<int64_t>(args.tiles * (k / X_BK), ex.num_sms);
     return (flags & QLIN_DEBUG_GROUP_SUMS) ? launch_i8x<true>(tm_w, tm_act, args, grid, ex)
                                            : launch_i8x<false>(tm_w, tm_act, args, grid, ex);
   }
@@ -1076,6 +1177,8 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
   args.tiles_t = (t + BN - 1) / BN;
   args.tiles = args.tiles_t * ((n + BM - 1) / BM);
   args.y_dtype = y_dtype;
+  args.partials = nullptr;
+  args.counters = nullptr;
   const bool debug = (flags & QLIN_DEBUG_GROUP_SUMS) != 0;
   const int grid = (int)std::min<int64_t>(args.tiles, ex.num_sms);
   switch (bits) {
