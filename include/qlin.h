@@ -216,9 +216,12 @@ QLIN_API int qlin_gemv(const qlin_weights* w, const uint16_t* x_bf16, int64_t t,
 /* Workspace bytes qlin_gemm_a8 should get for T tokens against an N x K
  * matrix: the activation codes and scales (T*K + T*K/64*4 bytes, 256-byte
  * aligned; the least a call with x_bf16 accepts) plus the weights expanded to
- * int8 once per call (N*K bytes).  With the full size the GEMM reads int8
- * weights through TMA (the faster kernel); with less, or none when the
- * activations come pre-quantized, it expands the codes on chip. */
+ * int8 once per call (N*K bytes) and the split-tile counters and FP32 partial
+ * tiles of its stream-K schedule (64 bytes per 128x128 tile and 128 KB per SM
+ * of the current device; sized for 256 SMs when no device is visible).  With
+ * the full size the GEMM reads int8 weights through TMA (the faster kernel);
+ * with less, or none when the activations come pre-quantized, it expands the
+ * codes on chip.  No part of it needs to be zero-filled. */
 QLIN_API int qlin_gemm_a8_workspace_bytes(int64_t t, int64_t n, int64_t k, size_t* bytes);
 
 /* Int8-route projection (prefill).  Weights must be Q3_G64, Q4_G64, Q5_G64 or Q6_G64
