@@ -667,6 +667,7 @@ struct __align__(1024) XStage {
   __half wsb[BM * 2];       // weight scales [row][group]
 };
 constexpr int X_NS = 6;
+constexpr int X_SK_MAX_WAVES = 8;           // stream-K for the last wave only below this many waves
 struct XSmem {
   XStage st[X_NS];
   uint64_t full[X_NS], empty[X_NS];
@@ -712,7 +713,7 @@ __global__ void expand_i8_kernel(const uint8_t* __restrict__ codes, const uint8_
   }
 }
 
-template <bool DEBUG>
+template <bool DEBUG, bool SK>
 __global__ void __launch_bounds__(X_THREADS, 1)
     gemm_i8x_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_act,
                     GemmArgs args) {
@@ -727,8 +728,12 @@ __global__ void __launch_bounds__(X_THREADS, 1)
   // their (tile, K chunk) iterations (stream-K), so that no SM idles through a
   // partial last wave.
   // (32-bit counts: tiles x chunks < 2^31 is checked on the host)
+  // SK = false (eight or more full waves: the idle part of the last one is
+  // small, and splitting it costs about as much): every tile whole, round
+  // robin, this CTA's rounds including the last, partial wave.
   const int P = (int)gridDim.x, ntiles = (int)args.tiles;
-  const int rounds = ntiles / P, dp_tiles = rounds * P;
+  const int rounds = SK ? ntiles / P : (ntiles - (int)blockIdx.x + P - 1) / P;
+  const int dp_tiles = SK ? rounds * P : ntiles;
   const int iters = (ntiles - dp_tiles) * nchunks;  // stream-K iterations
   const int it0 = (int)((int64_t)blockIdx.x * iters / P), it1 = (int)(((int64_t)blockIdx.x + 1) * iters / P);
   const int dp_jobs = rounds * nchunks;
@@ -942,7 +947,7 @@ __global__ void __launch_bounds__(X_THREADS, 1)
     }
     // the stream-K range: segments of whole tiles, or the first and last tile
     // of the range shared with neighbouring CTAs
-    for (int g = it0; g < it1 && ok;) {
+    for (int g = it0; SK && g < it1 && ok;) {
       const int tile = dp_tiles + g / nchunks;
       const int kc0 = g - (g / nchunks) * nchunks;
       const int kc1 = min(nchunks, kc0 + (it1 - g));
@@ -1064,11 +1069,11 @@ static int launch_a8(const CUtensorMap& tm_codes, const CUtensorMap& tm_hib, con
   return cuda_status(cudaLaunchKernelEx(&cfg, gemm_a8_kernel<BITS, DEBUG>, tm_codes, tm_hib, tm_act, args));
 }
 
-template <bool DEBUG>
+template <bool DEBUG, bool SK>
 static int launch_i8x(const CUtensorMap& tm_w, const CUtensorMap& tm_act, const GemmArgs& args, int grid,
                       const Exec& ex) {
   const size_t smem = sizeof(XSmem) + 1024;
-  const cudaError_t e0 = set_smem_once<gemm_i8x_kernel<DEBUG>>((int)smem);
+  const cudaError_t e0 = set_smem_once<gemm_i8x_kernel<DEBUG, SK>>((int)smem);
   if (e0 != cudaSuccess) return cuda_status(e0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -1080,7 +1085,7 @@ static int launch_i8x(const CUtensorMap& tm_w, const CUtensorMap& tm_act, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, gemm_i8x_kernel<DEBUG>, tm_w, tm_act, args));
+  return cuda_status(cudaLaunchKernelEx(&cfg, gemm_i8x_kernel<DEBUG, SK>, tm_w, tm_act, args));
 }
 
 int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, const float* xs,
@@ -1143,8 +1148,11 @@ int launch_gemm_a8(const qlin_weights& w, const uint16_t* x, const int8_t* xq, c
     args.counters = (int*)((uint8_t*)ex.workspace + wl.counters);
     // stream-K: every SM takes an equal share of the (tile, K chunk) iterations
     const int grid = (int)std::min<int64_t>(args.tiles * (k / X_BK), ex.num_sms);
-    return (flags & QLIN_DEBUG_GROUP_SUMS) ? launch_i8x<true>(tm_w, tm_act, args, grid, ex)
-                                           : launch_i8x<false>(tm_w, tm_act, args, grid, ex);
+    // stream-K for the tail only below X_SK_MAX_WAVES full waves
+    const bool sk = args.tiles < (int64_t)X_SK_MAX_WAVES * grid;
+    if (flags & QLIN_DEBUG_GROUP_SUMS)
+      return sk ? launch_i8x<true, true>(tm_w, tm_act, args, grid, ex) : launch_i8x<true, false>(tm_w, tm_act, args, grid, ex);
+    return sk ? launch_i8x<false, true>(tm_w, tm_act, args, grid, ex) : launch_i8x<false, false>(tm_w, tm_act, args, grid, ex);
   }
   // code plane: 128-byte swizzled nibble rows, or (Q3) unswizzled 64-byte crumb rows per stage
   const uint64_t crow = (uint64_t)(bits == 3 ? k / 4 : k / 2);
