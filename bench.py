@@ -52,6 +52,7 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     p.add_argument("--case", default=None,
                    help="run one kernel case only (for profilers): gemv:<q3|q4|q5|q6|q8|fp8|bf16>:<N>x<K>:T<t> "
+                        "or gemm_fp8:<N>x<K>:T<t> "
                         "or gemm_a8:<q3|q4|q5|q6>:<N>x<K>:T<t> or quantize:<T>x<K> or decode:<R>x<C>")
     return p.parse_args()
 
@@ -736,6 +737,15 @@ def run_case(args):
             ws.ensure(q.qlin_gemm_a8_workspace_bytes(t, n, k))
             fn = lambda: q.qlin_gemm_a8(pw, y, x=x, workspace=ws)  # noqa: E731
             units, unit = 2 * t * n * k, "TOPS"
+    elif kind == "gemm_fp8":
+        n, k = (int(v) for v in parts[1].split("x"))
+        t = int(parts[2][1:])
+        pw = packed(q, synth, q.FP8_ROW, n, k, 1, dev)
+        x = synth.activations_bf16(t, k, seed=2, device=dev)
+        y = torch.empty(t, n, dtype=torch.bfloat16, device=dev)
+        ws.ensure(q.qlin_gemm_fp8_workspace_bytes(t, k))
+        fn = lambda: q.qlin_gemm_fp8(pw, y, x=x, workspace=ws)  # noqa: E731
+        units, unit = 2 * t * n * k, "TFLOP/s"
     elif kind == "quantize":
         t, k = (int(v) for v in parts[1].split("x"))
         x = synth.activations_bf16(t, k, seed=2, device=dev)
