@@ -6,11 +6,16 @@
 //
 // B200 design:
 //   * quantize_act_kernel: eight lanes per (token, 64-group), 16-byte loads
-//     (two per thread in flight); amax by shuffles, the scale by IEEE
-//     division, the codes rint(x / scale) through the correctly rounded
-//     reciprocal with the IEEE division taking over near a half-integer
-//     (bit-identical to one division per element, see code_fast).
-//   * gemm_a8_kernel: persistent, one CTA per SM walking 128-row x 128-token
+//     (two per thread in flight, and the next two); amax by shuffles, the
+//     scale by IEEE division, the codes rint(x / scale) through the correctly
+//     rounded reciprocal with the IEEE division taking over near a
+//     half-integer (bit-identical to one division per element, see
+//     code_fast).
+//   * with the full workspace: expand_i8_kernel writes the weights as int8
+//     once per call and gemm_i8x_kernel (below) runs SS-operand integer MMAs
+//     fed by TMA, y in registers, full waves of tiles then a stream-K tail;
+//   * with only the activation part of the workspace:
+//     gemm_a8_kernel: persistent, one CTA per SM walking 128-row x 128-token
 //     tiles (neighbouring CTAs share weight rows; the activations stay in L2):
 //       - a TMA warp streams the packed weight codes, the int8 activation codes
 //         and (Q5) the high-bit plane into a 4-stage ring of 256-column chunks
@@ -636,7 +641,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 //                     (one thread per (row, 64-group), bandwidth-bound);
 //   gemm_i8x_kernel   persistent CTAs over 128-row x 128-token tiles, row-tile
 //                     major (consecutive CTAs share a weight tile, which L2
-//                     then serves):
+//                     then serves); with fewer than X_SK_MAX_WAVES full waves
+//                     of tiles, the tiles after the last full wave are split
+//                     over all CTAs by their K chunks (stream-K, SK = true):
 //     warp 0     TMA: per stage a 128 x 128 B box of int8 weights and one of
 //                int8 activation codes (two 64-groups, 128-byte swizzle); its
 //                lanes cp.async the stage's weight and activation scales;
